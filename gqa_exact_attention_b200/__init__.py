@@ -1,0 +1,139 @@
+"""Exact grouped-query attention forward on B200 (sm_100a): Python binding.
+
+Argument marshalling only: every step of the computation runs in the CUDA kernels of
+``libgqa_attn.so`` (built in-tree from ``csrc/``).  PyTorch supplies device memory and
+the current stream.  There is no fallback: if the library cannot be loaded, the calls
+raise.
+
+The C contract is ``include/gqa_attn.h``; the names here are the same.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes", "gqa_attn_status_string",
+    "gqa_attn_device_status", "GqaError", "lib_path", "load",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libgqa_attn.so")
+
+GQA_OK = 0
+STATUS_NAMES = {
+    0: "GQA_OK", 1: "GQA_ERR_NULL", 2: "GQA_ERR_SHAPE", 3: "GQA_ERR_HEADS",
+    4: "GQA_ERR_HEADDIM", 5: "GQA_ERR_ALIGN", 6: "GQA_ERR_ARCH", 7: "GQA_ERR_ALLOC",
+    8: "GQA_ERR_CUDA", 9: "GQA_ERR_TIMEOUT",
+}
+
+
+class GqaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load():
+    """Load ``libgqa_attn.so`` (building it in-tree first if it is absent or stale and
+    nvcc is available).  Raises if it cannot be loaded."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    try:
+        from . import _build
+        if _build._stale() and _have_nvcc():
+            _build.build()
+    except Exception as e:  # a failed build must not hide behind an old library
+        if not os.path.exists(lib_path):
+            raise RuntimeError(f"libgqa_attn.so is missing and could not be built: {e}") from e
+    if not os.path.exists(lib_path):
+        raise RuntimeError(f"libgqa_attn.so not found at {lib_path}; run the package build")
+    L = ctypes.CDLL(lib_path)
+    i, f, p, sz = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+    L.gqa_attn_fwd.argtypes = [p, p, p, p, p, i, i, i, i, i, i, f, i, i, i, p]
+    L.gqa_attn_fwd.restype = i
+    L.gqa_attn_choose.argtypes = [i, i, i, i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(i)]
+    L.gqa_attn_choose.restype = i
+    L.gqa_attn_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i, i]
+    L.gqa_attn_workspace_bytes.restype = sz
+    L.gqa_attn_status_string.argtypes = [i]
+    L.gqa_attn_status_string.restype = ctypes.c_char_p
+    L.gqa_attn_device_status.argtypes = [i]
+    L.gqa_attn_device_status.restype = i
+    _lib = L
+    return L
+
+
+def _have_nvcc() -> bool:
+    from shutil import which
+    return which("nvcc") is not None
+
+
+def gqa_attn_status_string(status: int) -> str:
+    return load().gqa_attn_status_string(int(status)).decode()
+
+
+def _check(status: int):
+    if status != GQA_OK:
+        raise GqaError(status, gqa_attn_status_string(status))
+
+
+def gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, causal, num_sms=148):
+    """The heuristic's (pack_gqa, num_splits) for this shape (host only)."""
+    pk, ns = ctypes.c_int(), ctypes.c_int()
+    _check(load().gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, int(bool(causal)), num_sms,
+                                  ctypes.byref(pk), ctypes.byref(ns)))
+    return pk.value, ns.value
+
+
+def gqa_attn_workspace_bytes(B, Sq, Sk, Hq, Hk, d, causal, pack_gqa=-1, num_splits=0):
+    return int(load().gqa_attn_workspace_bytes(B, Sq, Sk, Hq, Hk, d, int(bool(causal)),
+                                               pack_gqa, num_splits))
+
+
+def gqa_attn_device_status(reset: bool = False) -> int:
+    """The device status word (0 = ok, 9 = a bounded wait timed out); synchronous."""
+    return int(load().gqa_attn_device_status(int(bool(reset))))
+
+
+def gqa_attn_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, pack_gqa=-1,
+                 num_splits=0, stream=None):
+    """out, lse = gqa_attn_fwd(q, k, v, ...) on the current CUDA stream.
+
+    q: bf16 [B, Sq, Hq, d]; k, v: bf16 [B, Sk, Hk, d]; all contiguous CUDA tensors.
+    out: fp32 [B, Sq, Hq, d] and lse: fp32 [B, Hq, Sq] are allocated when not given.
+    scale defaults to 1/sqrt(d).
+    """
+    import torch
+
+    B, Sq, Hq, d = q.shape
+    Sk, Hk = k.shape[1], k.shape[2]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Sk, Hk, d] matching q")
+    if out is None:
+        out = torch.empty((B, Sq, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    for name, t in (("out", out), ("lse", lse)):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous fp32 tensor on q's device")
+    if tuple(out.shape) != (B, Sq, Hq, d) or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("out must be [B, Sq, Hq, d] and lse [B, Hq, Sq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        _check(load().gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), B, Sq, Sk, Hq, Hk, d, float(scale),
+                                   int(bool(causal)), int(pack_gqa), int(num_splits),
+                                   stream.cuda_stream))
+    return out, lse

@@ -1,0 +1,318 @@
+// C ABI of libgqa_attn.so: argument validation, the pack/split heuristic, TMA tensor
+// maps, split-KV scratch and kernel launches.  See include/gqa_attn.h for the contract.
+#include "gqa_attn.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "fwd_params.h"
+#include "launch.h"
+
+namespace {
+
+using gqa::kBlockM;
+using gqa::kBlockN;
+using gqa::kMaxSplits;
+
+constexpr int kDefaultSms = 148;
+
+struct Plan {
+    int pack;        // 0 / 1
+    int nt;          // tiles per CTA unit (1 or 2)
+    int pos_per_tile;
+    int rows_valid;
+    int n_hg;
+    int n_mt;
+    int splits;      // resolved, clamped
+    int kv_blocks;
+    long long units;
+};
+
+int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+gqa_status validate_shape(int B, int Sq, int Sk, int Hq, int Hk, int d, int pack, int splits) {
+    if (B < 1 || Sq < 1 || Sk < 1 || Hq < 1 || Hk < 1) return GQA_ERR_SHAPE;
+    if (pack < -1 || pack > 1 || splits < 0) return GQA_ERR_SHAPE;
+    if (Hq % Hk != 0) return GQA_ERR_HEADS;
+    if (d != 64 && d != 128) return GQA_ERR_HEADDIM;
+    if (pack == 1 && Hq / Hk > kBlockM) return GQA_ERR_SHAPE;  // one position must fit a tile
+    // TMA coordinates and in-kernel row indices are 32-bit
+    const long long rows_out = (long long)B * Hq * Sq;
+    if (rows_out >= (1ll << 31) || (long long)B * Sk * Hk >= (1ll << 31)) return GQA_ERR_SHAPE;
+    return GQA_OK;
+}
+
+// Padded tile rows computed per kv group with and without packing.
+void padded_rows(int Sq, int g, long long* unpacked, long long* packed) {
+    *unpacked = (long long)g * ceil_div(Sq, kBlockM) * kBlockM;
+    const int P = kBlockM / g;
+    *packed = P >= 1 ? (long long)ceil_div(Sq, P) * kBlockM : (1ll << 62);
+}
+
+int choose_pack(int Sq, int Hq, int Hk) {
+    const int g = Hq / Hk;
+    if (g == 1 || g > kBlockM) return 0;
+    long long un, pk;
+    padded_rows(Sq, g, &un, &pk);
+    return pk < un ? 1 : 0;
+}
+
+// Fill everything except the split count from the shape and the pack choice.
+Plan make_plan(int B, int Sq, int Sk, int Hq, int Hk, int pack) {
+    Plan pl{};
+    const int g = Hq / Hk;
+    pl.pack = pack;
+    pl.pos_per_tile = pack ? kBlockM / g : kBlockM;
+    pl.rows_valid = pack ? g * pl.pos_per_tile : kBlockM;
+    pl.n_hg = pack ? Hk : Hq;
+    const int tiles = ceil_div(Sq, pl.pos_per_tile);
+    pl.nt = tiles >= 2 ? 2 : 1;
+    pl.n_mt = ceil_div(tiles, pl.nt);
+    pl.kv_blocks = ceil_div(Sk, kBlockN);
+    pl.units = (long long)pl.n_mt * B * pl.n_hg;
+    (void)B;
+    return pl;
+}
+
+int choose_splits(const Plan& pl, int d, int num_sms) {
+    const int slots = num_sms * gqa::fwd_ctas_per_sm(d, pl.nt);
+    if (pl.units >= slots) return 1;
+    int s = ceil_div(slots, pl.units);
+    const int cap = pl.kv_blocks / 2 > 1 ? pl.kv_blocks / 2 : 1;
+    if (s > cap) s = cap;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return s < 1 ? 1 : s;
+}
+
+int clamp_splits(int s, int kv_blocks) {
+    if (s > kv_blocks) s = kv_blocks;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return s < 1 ? 1 : s;
+}
+
+Plan resolve(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal, int pack, int splits,
+             int num_sms) {
+    (void)causal;
+    if (pack < 0) pack = choose_pack(Sq, Hq, Hk);
+    Plan pl = make_plan(B, Sq, Sk, Hq, Hk, pack);
+    pl.splits = clamp_splits(splits <= 0 ? choose_splits(pl, d, num_sms) : splits, pl.kv_blocks);
+    pl.units *= pl.splits;
+    return pl;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encode_tiled() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor [B, S, H, d] as a 4-D map (d, H, S, B), 128-byte swizzle, zero fill out of
+// bounds, box (64, box_h, box_s, 1).
+bool encode_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, int box_h,
+                 int box_s) {
+    EncodeTiled enc = get_encode_tiled();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)S * H * d * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    int ok = 0;  // 1: sm_100
+};
+
+gqa_status device_info(int* dev_out, DeviceInfo* info) {
+    static DeviceInfo cache[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    *dev_out = dev;
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && cache[dev].sms > 0) {
+        *info = cache[dev];
+        return GQA_OK;
+    }
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    DeviceInfo di;
+    di.sms = sms;
+    di.ok = (major == 10 && minor == 0) ? 1 : 0;
+    if (dev >= 0 && dev < 64) cache[dev] = di;
+    *info = di;
+    return GQA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+long long timeout_ns() {
+    const char* e = std::getenv("GQA_WAIT_TIMEOUT_MS");
+    long long ms = e ? std::atoll(e) : 4000;
+    if (ms < 1) ms = 1;
+    return ms * 1000000ll;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gqa_attn_status_string(gqa_status s) {
+    switch (s) {
+        case GQA_OK: return "ok";
+        case GQA_ERR_NULL: return "a required pointer is NULL";
+        case GQA_ERR_SHAPE: return "invalid shape, pack_gqa or num_splits";
+        case GQA_ERR_HEADS: return "Hq is not a multiple of Hk";
+        case GQA_ERR_HEADDIM: return "head dim must be 64 or 128";
+        case GQA_ERR_ALIGN: return "pointers must be 16-byte aligned";
+        case GQA_ERR_ARCH: return "device is not sm_100 (B200 class)";
+        case GQA_ERR_ALLOC: return "split-KV workspace allocation failed";
+        case GQA_ERR_CUDA: return "CUDA call failed";
+        case GQA_ERR_TIMEOUT: return "an in-kernel bounded wait timed out";
+    }
+    return "unknown status";
+}
+
+gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal, int num_sms,
+                           int* pack_gqa, int* num_splits) {
+    if (!pack_gqa || !num_splits) return GQA_ERR_NULL;
+    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, -1, 0);
+    if (st != GQA_OK) return st;
+    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal, -1, 0, num_sms > 0 ? num_sms : kDefaultSms);
+    *pack_gqa = pl.pack;
+    *num_splits = pl.splits;
+    return GQA_OK;
+}
+
+size_t gqa_attn_workspace_bytes(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
+                                int pack_gqa, int num_splits) {
+    if (validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits) != GQA_OK) return 0;
+    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal, pack_gqa, num_splits, kDefaultSms);
+    if (pl.splits <= 1) return 0;
+    const size_t rows = (size_t)B * Hq * Sq;
+    return (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
+}
+
+gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out, float* lse,
+                        int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
+                        int pack_gqa, int num_splits, void* stream_ptr) {
+    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
+    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
+    if (st != GQA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+        return GQA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return GQA_ERR_SHAPE;
+    int dev = 0;
+    DeviceInfo info;
+    st = device_info(&dev, &info);
+    if (st != GQA_OK) return st;
+    if (!info.ok) return GQA_ERR_ARCH;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+
+    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms);
+    const int g = Hq / Hk;
+
+    gqa::FwdParams p{};
+    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM) ||
+        !encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
+        !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
+        return GQA_ERR_CUDA;
+    p.out = out;
+    p.lse = lse;
+    p.B = B;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.Hq = Hq;
+    p.Hk = Hk;
+    p.g = g;
+    p.pack = pl.pack;
+    p.pos_per_tile = pl.pos_per_tile;
+    p.rows_valid = pl.rows_valid;
+    p.causal = causal ? 1 : 0;
+    p.num_splits = pl.splits;
+    p.n_hg = pl.n_hg;
+    p.n_mt = pl.n_mt;
+    p.n_units = (int)pl.units;
+    p.kv_blocks = pl.kv_blocks;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.div_g = gqa::make_fastdiv((uint32_t)g);
+    p.status = nullptr;
+    p.timeout_ns = timeout_ns();
+
+    void* ws = nullptr;
+    if (pl.splits > 1) {
+        const size_t rows = (size_t)B * Hq * Sq;
+        const size_t bytes = (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
+        if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
+        if (cudaMallocAsync(&ws, bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GQA_ERR_ALLOC;
+        }
+        p.o_part = static_cast<float*>(ws);
+        p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
+    }
+
+    const int slots = info.sms * gqa::fwd_ctas_per_sm(d, pl.nt);
+    const int grid = (int)(pl.units < slots ? pl.units : slots);
+    if (gqa::launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) {
+        if (ws) cudaFreeAsync(ws, stream);
+        return GQA_ERR_CUDA;
+    }
+    if (pl.splits > 1) {
+        gqa::CombineParams c{};
+        c.o_part = p.o_part;
+        c.lse_part = p.lse_part;
+        c.out = out;
+        c.lse = lse;
+        c.B = B;
+        c.Sq = Sq;
+        c.Hq = Hq;
+        c.num_splits = pl.splits;
+        cudaError_t e = gqa::launch_combine(c, d, info.sms, stream);
+        cudaFreeAsync(ws, stream);
+        if (e != cudaSuccess) return GQA_ERR_CUDA;
+    }
+    return GQA_OK;
+}
+
+gqa_status gqa_attn_device_status(int reset) {
+    unsigned int* ptr = gqa::device_status_symbol();
+    if (!ptr) return GQA_ERR_CUDA;
+    unsigned int h = 0;
+    if (cudaMemcpy(&h, ptr, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return GQA_ERR_CUDA;
+    if (reset) {
+        unsigned int z = 0;
+        if (cudaMemcpy(ptr, &z, sizeof(z), cudaMemcpyHostToDevice) != cudaSuccess)
+            return GQA_ERR_CUDA;
+    }
+    return h ? GQA_ERR_TIMEOUT : GQA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Parameters shared by the host plan (api.cpp) and the sm_100a kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "fast_divmod.h"
+
+namespace gqa {
+
+constexpr int kBlockM = 128;  // rows of one tile (the tcgen05 M)
+constexpr int kBlockN = 128;  // keys of one K/V block
+constexpr int kMaxSplits = 16;
+
+// Work unit: one CTA-iteration of the persistent kernel covers NT consecutive tiles of
+// one (batch, head-or-group) pair, over one split of the key axis.
+struct FwdParams {
+    CUtensorMap tm_q;  // q as 4-D (d, Hq, Sq, B); box (64, g or 1, positions, 1)
+    CUtensorMap tm_k;  // k as 4-D (d, Hk, Sk, B); box (64, 1, 128, 1)
+    CUtensorMap tm_v;  // v likewise
+
+    float* out;       // [B, Sq, Hq, d]       (num_splits == 1)
+    float* lse;       // [B, Hq, Sq]          (num_splits == 1)
+    float* o_part;    // [splits, B, Hq, Sq, d] (num_splits > 1)
+    float* lse_part;  // [splits, B, Hq, Sq]    (num_splits > 1)
+
+    int B, Sq, Sk, Hq, Hk;
+    int g;             // Hq / Hk
+    int pack;          // 1: a tile holds g heads x pos_per_tile positions
+    int pos_per_tile;  // positions one tile covers (packed: floor(128/g); else 128)
+    int rows_valid;    // rows of a tile that map to (position, head) (packed: g*pos_per_tile)
+    int causal;
+    int num_splits;
+    int n_hg;          // heads-or-groups per batch: Hq (unpacked) or Hk (packed)
+    int n_mt;          // CTA-units along the query axis per (b, hg)
+    int n_units;       // n_mt * B * n_hg * num_splits
+    int kv_blocks;     // ceil(Sk / 128)
+    float scale_log2;  // scale * log2(e)
+    FastDiv div_g;     // row -> (position, head-in-group) for packed tiles
+    unsigned int* status;  // status word for bounded-wait timeouts (NULL: the library's own)
+    long long timeout_ns;  // limit of each in-kernel wait
+};
+
+struct CombineParams {
+    const float* o_part;
+    const float* lse_part;
+    float* out;
+    float* lse;
+    int B, Sq, Hq, num_splits;
+};
+
+}  // namespace gqa

@@ -1,0 +1,623 @@
+// Exact GQA attention forward for sm_100a: persistent, warp-specialised, TMA + tcgen05.
+//
+// One CTA runs on one SM and walks a static stride of work units.  A unit is NT
+// consecutive 128-row query tiles of one (batch, head) pair (or, with PackGQA, of one
+// (batch, kv-group) pair whose g query heads are folded into the rows), over one
+// split of the key axis.  Roles:
+//   warp 0        TMA producer: Q tiles once per unit, then a ring of K/V blocks.
+//   warp 1        MMA issuer (one thread): S_t = Q_t K^T into TMEM (both operands in
+//                 shared memory), then O_t += P_t V with P_t read from TMEM.
+//   warps 2..     NT softmax warpgroups, one per tile; thread = tile row = TMEM lane.
+//                 Each reads its S row from TMEM, masks (causal, key tail), keeps the
+//                 running max / sum, writes P (bf16) over S in TMEM, rescales O in TMEM
+//                 when the max grows, and runs the epilogue (O / l, LSE).
+//
+// The computation follows the scaled dot-product attention definition
+// ("PyTorch 性能分析深度指南 (第三部分)", section "Attention 的计算挑战") with the GQA head
+// sharing of "优化GQA在Flash-Attention中的批量敏感性" (section "分组查询注意力的核心设计"),
+// the PackGQA row folding of the same page (section "Flash-Attention的PackGQA优化") and
+// the split-KV partials of "為什么 GQA 推理吞吐先升后降…4 步速查" (section "修復").
+// The online softmax (running max with deferred rescaling) is the standard exact
+// reformulation of the row softmax; it reaches the definition up to fp32 rounding.
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+
+#include "fwd_params.h"
+#include "launch.h"
+#include "ptx_sm100.cuh"
+
+namespace gqa {
+
+__device__ unsigned int g_device_status = 0;
+
+namespace {
+
+using namespace ptx;
+
+template <int HD, int NT>
+struct FwdCfg {
+    static constexpr int kChunks = HD / 64;              // 128-byte column chunks of a row
+    static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 bytes
+    static constexpr int kTileBytes = kChunks * kChunkBytes;
+    static constexpr int kSlots = (NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 2 : 4);
+    static constexpr int kSoftmaxWarps = 4 * NT;
+    static constexpr int kThreads = (2 + kSoftmaxWarps) * 32;
+    static constexpr int kCtasPerSm = (NT == 2) ? 1 : 2;
+    static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
+    static constexpr int kNumBars = 2 * kSlots + 6 * NT + 1;
+    static constexpr int kSmemBytes =
+        1024 /* alignment slack */ + NT * kTileBytes + kSlots * kTileBytes + 8 * kNumBars + 16;
+    static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, HD, true);
+    __host__ __device__ static constexpr int s_col(int t) { return t * 128; }
+    __host__ __device__ static constexpr int o_col(int t) { return NT * 128 + t * HD; }
+};
+
+// Geometry of one work unit, computed identically by every role.
+template <int NT>
+struct UnitGeom {
+    int b, hg, split, kvh;
+    int pos0[NT];   // first query position of tile t
+    int n[NT];      // key blocks tile t processes in this split
+    int kb_lo;      // first key block of the split
+    int nblk;       // max over tiles of n[t]
+};
+
+template <int NT>
+__device__ __forceinline__ UnitGeom<NT> unit_geom(int u, const FwdParams& p) {
+    UnitGeom<NT> g;
+    g.split = u % p.num_splits;
+    u /= p.num_splits;
+    g.hg = u % p.n_hg;
+    u /= p.n_hg;
+    g.b = u % p.B;
+    u /= p.B;
+    const int mt = p.n_mt - 1 - u;  // longest (latest-position) units first
+    g.kvh = p.pack ? g.hg : g.hg / p.g;
+    int kb_end[NT];
+    int kb_union = 0;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        g.pos0[t] = (mt * NT + t) * p.pos_per_tile;
+        kb_end[t] = 0;
+        if (g.pos0[t] < p.Sq) {
+            int last = min(g.pos0[t] + p.pos_per_tile, p.Sq) - 1;
+            int key_end = p.Sk;
+            if (p.causal) key_end = max(0, min(p.Sk, last + 1 + (p.Sk - p.Sq)));
+            kb_end[t] = (key_end + kBlockN - 1) / kBlockN;
+        }
+        kb_union = max(kb_union, kb_end[t]);
+    }
+    g.kb_lo = (int)(((long long)g.split * kb_union) / p.num_splits);
+    const int kb_hi = (int)(((long long)(g.split + 1) * kb_union) / p.num_splits);
+    g.nblk = 0;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        g.n[t] = max(0, min(kb_hi, kb_end[t]) - g.kb_lo);
+        g.nblk = max(g.nblk, g.n[t]);
+    }
+    return g;
+}
+
+// a[t] for a run-time t without dynamic indexing (keeps the arrays in registers)
+template <int NT>
+__device__ __forceinline__ int pick(const int (&a)[NT], int t) {
+    int v = a[0];
+#pragma unroll
+    for (int i = 1; i < NT; ++i) v = (t == i) ? a[i] : v;
+    return v;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting or when
+// this wait ran past the time limit (then it records the timeout and starts the abort).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile uint32_t* abort_flag,
+                                             const FwdParams& p) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer();
+    uint32_t spins = 0;
+    while (!mbar_try_wait(bar, parity)) {
+        if ((++spins & 255u) == 0) {
+            if (*abort_flag) return false;
+            if ((long long)(globaltimer() - t0) > p.timeout_ns) {
+                *abort_flag = 1u;
+                atomicOr(p.status ? p.status : &g_device_status, 1u);
+                return false;
+            }
+        }
+    }
+    return true;
+}
+
+// Wait used during teardown: ignores the abort flag, gives up silently at the limit.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const FwdParams& p) {
+    uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if ((long long)(globaltimer() - t0) > p.timeout_ns) return;
+    }
+}
+
+template <int HD, int NT>
+__global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCtasPerSm)
+    gqa_fwd_kernel(const __grid_constant__ FwdParams p) {
+    using C = FwdCfg<HD, NT>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw);
+
+    const uint32_t sQ = base;
+    const uint32_t sKV = base + NT * C::kTileBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NT * C::kTileBytes + C::kSlots * C::kTileBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const uint32_t bar0 = smem_u32(bars);
+    auto kv_full = [&](int s) { return bar0 + 8u * s; };
+    auto kv_empty = [&](int s) { return bar0 + 8u * (C::kSlots + s); };
+    auto q_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + t); };
+    auto q_empty = [&](int t) { return bar0 + 8u * (2 * C::kSlots + NT + t); };
+    auto s_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 2 * NT + t); };
+    auto p_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 3 * NT + t); };
+    auto o_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 4 * NT + t); };
+    auto o_empty = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 5 * NT + t); };
+    const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 6 * NT);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(kv_full(s), 1);
+            mbar_init(kv_empty(s), 1);
+        }
+        for (int t = 0; t < NT; ++t) {
+            mbar_init(q_full(t), 1);
+            mbar_init(q_empty(t), 1);
+            mbar_init(s_full(t), 1);
+            mbar_init(p_full(t), 128);
+            mbar_init(o_full(t), 1);
+            mbar_init(o_empty(t), 128);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc<C::kTmemCols>(smem_u32(tmem_slot));
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
+            uint32_t qn[NT] = {};  // Q loads issued per tile
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const UnitGeom<NT> g = unit_geom<NT>(u, p);
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (g.n[t] == 0 || !ok) continue;
+                    if (qn[t] > 0) ok = wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p);
+                    if (!ok) break;
+                    const int rows = p.pack ? p.rows_valid : kBlockM;
+                    mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
+                    const int hcoord = p.pack ? g.hg * p.g : g.hg;
+#pragma unroll
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, q_full(t),
+                                    c * 64, hcoord, g.pos0[t], g.b);
+                    ++qn[t];
+                }
+                for (int it = 0; it < g.nblk && ok; ++it) {
+                    const int kpos = (g.kb_lo + it) * kBlockN;
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        const int slot = ld % C::kSlots;
+                        if (ld >= (uint32_t)C::kSlots)
+                            ok = wait_bounded(kv_empty(slot), ((ld / C::kSlots) - 1) & 1u, abort_flag, p);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(kv_full(slot), (uint32_t)C::kTileBytes);
+#pragma unroll
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes,
+                                        w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v,
+                                        kv_full(slot), c * 64, g.kvh, kpos, g.b);
+                        ++ld;
+                    }
+                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA's memory is released
+                const uint32_t first = ld > (uint32_t)C::kSlots ? ld - C::kSlots : 0u;
+                for (uint32_t l = first; l < ld; ++l)
+                    wait_drain(kv_full(l % C::kSlots), (l / C::kSlots) & 1u, p);
+                for (int t = 0; t < NT; ++t)
+                    if (qn[t] > 0) wait_drain(q_full(t), (qn[t] - 1) & 1u, p);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t ld = 0;
+            uint32_t qn[NT] = {}, pn[NT] = {}, on[NT] = {};
+            bool ok = true;
+
+            auto issue_s = [&](int t, int slot) {
+                const uint32_t a0 = sQ + t * C::kTileBytes;
+                const uint32_t b0 = sKV + slot * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                    mma_ss(tmem + C::s_col(t), sdesc_sw128(a0 + off, 16, 1024),
+                           sdesc_sw128(b0 + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int t, int slot, bool accumulate) {
+                const uint32_t b0 = sKV + slot * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                    mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                           sdesc_sw128(b0 + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
+                           (accumulate || kk > 0) ? 1u : 0u);
+            };
+
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const UnitGeom<NT> g = unit_geom<NT>(u, p);
+                if (g.nblk == 0) continue;
+                // first key block: S_t for every tile that has keys
+                int slot_k = ld % C::kSlots;
+                ok = wait_bounded(kv_full(slot_k), (ld / C::kSlots) & 1u, abort_flag, p);
+                if (!ok) break;
+                ++ld;
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (g.n[t] == 0 || !ok) continue;
+                    ok = wait_bounded(q_full(t), qn[t] & 1u, abort_flag, p);
+                    if (!ok) break;
+                    ++qn[t];
+                    tc_fence_after();
+                    issue_s(t, slot_k);
+                    mma_commit(s_full(t));
+                    if (g.n[t] == 1) mma_commit(q_empty(t));
+                }
+                if (!ok) break;
+                mma_commit(kv_empty(slot_k));
+
+                for (int it = 0; it < g.nblk && ok; ++it) {
+                    const int slot_v = ld % C::kSlots;
+                    ok = wait_bounded(kv_full(slot_v), (ld / C::kSlots) & 1u, abort_flag, p);
+                    if (!ok) break;
+                    ++ld;
+                    // K of the next block: waited for only when its first S is issued
+                    const bool next = it + 1 < g.nblk;
+                    const uint32_t ld_n = ld;
+                    const int slot_n = ld_n % C::kSlots;
+                    bool k_ready = false;
+                    if (next) ++ld;
+                    tc_fence_after();
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        if (it >= g.n[t] || !ok) continue;
+                        ok = wait_bounded(p_full(t), pn[t] & 1u, abort_flag, p);
+                        if (!ok) break;
+                        ++pn[t];
+                        if (it == 0 && on[t] > 0) {
+                            // the previous unit's epilogue must have read O_t out
+                            ok = wait_bounded(o_empty(t), (on[t] - 1) & 1u, abort_flag, p);
+                            if (!ok) break;
+                        }
+                        tc_fence_after();
+                        issue_pv(t, slot_v, it > 0);
+                        if (it + 1 < g.n[t]) {
+                            if (!k_ready) {
+                                ok = wait_bounded(kv_full(slot_n), (ld_n / C::kSlots) & 1u, abort_flag, p);
+                                if (!ok) break;
+                                k_ready = true;
+                                tc_fence_after();
+                            }
+                            issue_s(t, slot_n);
+                            mma_commit(s_full(t));
+                            if (it + 2 == g.n[t]) mma_commit(q_empty(t));
+                        } else {
+                            mma_commit(o_full(t));
+                            ++on[t];
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit(kv_empty(slot_v));
+                    if (next) mma_commit(kv_empty(slot_n));
+                }
+            }
+            // every MMA issued so far must be complete before TMEM is released
+            mma_commit(mma_done);
+            wait_drain(mma_done, 0u, p);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = (warp - 2) >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t s_addr = tl + C::s_col(t);
+        const uint32_t o_addr = tl + C::o_col(t);
+        uint32_t sn = 0, on = 0;
+        bool ok = true;
+        const float kNegInf = -INFINITY;
+        constexpr float kLn2 = 0.69314718055994530942f;
+
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+            const UnitGeom<NT> g = unit_geom<NT>(u, p);
+            const int n_t = pick<NT>(g.n, t);
+            const int pos0_t = pick<NT>(g.pos0, t);
+            // row -> (position, head)
+            int pos, head;
+            bool row_ok;
+            if (p.pack) {
+                uint32_t pr, hh;
+                fastdivmod((uint32_t)row, p.div_g, pr, hh);
+                pos = pos0_t + (int)pr;
+                head = g.hg * p.g + (int)hh;
+                row_ok = row < p.rows_valid && pos < p.Sq;
+            } else {
+                pos = pos0_t + row;
+                head = g.hg;
+                row_ok = pos < p.Sq;
+            }
+            // exclusive key bound of this row (causal: j <= pos + Sk - Sq)
+            const int kmax = p.causal ? min(p.Sk, pos + 1 + (p.Sk - p.Sq)) : p.Sk;
+
+            float m = kNegInf;  // reference max, log2 units
+            float l = 0.f;
+            for (int it = 0; it < n_t; ++it) {
+                ok = __all_sync(0xffffffffu, wait_bounded(s_full(t), sn & 1u, abort_flag, p));
+                if (!ok) break;
+                ++sn;
+                tc_fence_after();
+                float s[128];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(s_addr + c * 32, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                }
+                tmem_wait_ld();
+                // scores in log2 units, then masking
+#pragma unroll
+                for (int i = 0; i < 128; ++i) s[i] *= p.scale_log2;
+                const int lim = kmax - (g.kb_lo + it) * kBlockN;
+                if (lim < kBlockN) {
+#pragma unroll
+                    for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : kNegInf;
+                }
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int i = 4; i < 128; i += 4) {
+                    mx0 = fmaxf(mx0, s[i]);
+                    mx1 = fmaxf(mx1, s[i + 1]);
+                    mx2 = fmaxf(mx2, s[i + 2]);
+                    mx3 = fmaxf(mx3, s[i + 3]);
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                // Deferred rescaling: move the reference max only when the block's max
+                // exceeds it by more than 8 (a factor 256), which keeps every p <= 256.
+                const bool grow = mx > m + 8.0f;  // false when mx = -inf; true when m = -inf < mx
+                float alpha = 1.f;
+                if (grow) {
+                    alpha = (m == kNegInf) ? 0.f : ex2_approx(m - mx);
+                    l *= alpha;
+                    m = mx;
+                }
+                // P = exp2(t - m) as bf16, written over S in TMEM (S is already in registers)
+                const float m_use = (m == kNegInf) ? 0.f : m;
+                float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = ex2_approx(s[c * 32 + 2 * i] - m_use);
+                        const float p1 = ex2_approx(s[c * 32 + 2 * i + 1] - m_use);
+                        ls0 += p0;
+                        ls1 += p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(s_addr + c * 16, pk);
+                }
+                l += ls0 + ls1;
+                // O rescale (after P, so the S registers are free): PV of the previous
+                // block is complete, because this block's S was issued after it.
+                if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t r[32];
+                        tmem_ld32(o_addr + c * 32, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st32(o_addr + c * 32, r);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(p_full(t));
+            }
+            if (!ok) break;
+
+            // ---------------------------------------------------------- epilogue
+            const bool has = n_t > 0;
+            if (has) {
+                ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), on & 1u, abort_flag, p));
+                if (!ok) break;
+                ++on;
+                tc_fence_after();
+            }
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : kNegInf;
+            float* orow;
+            float* lrow;
+            if (p.num_splits == 1) {
+                orow = p.out + (((size_t)g.b * p.Sq + pos) * p.Hq + head) * HD;
+                lrow = p.lse + ((size_t)g.b * p.Hq + head) * p.Sq + pos;
+            } else {
+                const size_t r = (((size_t)g.split * p.B + g.b) * p.Hq + head) * p.Sq + pos;
+                orow = p.o_part + r * HD;
+                lrow = p.lse_part + r;
+            }
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t r[32];
+                if (has) {
+                    tmem_ld32(o_addr + c * 32, r);
+                    tmem_wait_ld();
+                }
+                if (row_ok) {
+                    float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        float4 v;
+                        v.x = has ? __uint_as_float(r[4 * i + 0]) * inv_l : 0.f;
+                        v.y = has ? __uint_as_float(r[4 * i + 1]) * inv_l : 0.f;
+                        v.z = has ? __uint_as_float(r[4 * i + 2]) * inv_l : 0.f;
+                        v.w = has ? __uint_as_float(r[4 * i + 3]) * inv_l : 0.f;
+                        dst[i] = v;
+                    }
+                }
+            }
+            if (row_ok) *lrow = lse_v;
+            if (has) {
+                tc_fence_before();
+                mbar_arrive(o_empty(t));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc<C::kTmemCols>(tmem);
+    }
+}
+
+// ---------------------------------------------------------------- split-KV combine
+// One warp per output row (b, h, i): M = max_s lse_s, w_s = exp(lse_s - M),
+// lse = M + ln sum w_s, O = sum_s w_s O_s / sum_s w_s.
+template <int HD>
+__global__ void __launch_bounds__(256) gqa_combine_kernel(const CombineParams p) {
+    constexpr int kPer = HD / 32;
+    const long long rows = (long long)p.B * p.Hq * p.Sq;
+    const int lane = threadIdx.x & 31;
+    const long long warps_total = (long long)gridDim.x * (blockDim.x >> 5);
+    const float kNegInf = -INFINITY;
+    for (long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows;
+         r += warps_total) {
+        float ls = (lane < p.num_splits) ? p.lse_part[(long long)lane * rows + r] : kNegInf;
+        float M = ls;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float w = (M == kNegInf || ls == kNegInf) ? 0.f : __expf(ls - M);
+        float wsum = w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+        float acc[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+        for (int s = 0; s < p.num_splits; ++s) {
+            const float ws = __shfl_sync(0xffffffffu, w, s);
+            if (ws == 0.f) continue;
+            const float* src = p.o_part + ((long long)s * rows + r) * HD + lane * kPer;
+            if constexpr (kPer == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(src);
+                acc[0] += ws * v.x;
+                acc[1] += ws * v.y;
+                acc[2] += ws * v.z;
+                acc[3] += ws * v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(src);
+                acc[0] += ws * v.x;
+                acc[1] += ws * v.y;
+            }
+        }
+        const float inv = (wsum > 0.f) ? 1.f / wsum : 0.f;
+        // r = (b * Hq + h) * Sq + i  ->  out[b, i, h, :]
+        const long long i = r % p.Sq;
+        const long long bh = r / p.Sq;
+        const long long h = bh % p.Hq;
+        const long long b = bh / p.Hq;
+        float* dst = p.out + ((b * p.Sq + i) * p.Hq + h) * HD + lane * kPer;
+        if constexpr (kPer == 4) {
+            *reinterpret_cast<float4*>(dst) =
+                make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        } else {
+            *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+        }
+        if (lane == 0) p.lse[r] = (wsum > 0.f) ? M + __logf(wsum) : kNegInf;
+    }
+}
+
+template <int HD, int NT>
+cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
+    using C = FwdCfg<HD, NT>;
+    // the attribute is per device; setting it again is idempotent, so the race is benign
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gqa_fwd_kernel<HD, NT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    gqa_fwd_kernel<HD, NT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int fwd_ctas_per_sm(int hd, int nt) {
+    if (nt == 2) return hd == 128 ? FwdCfg<128, 2>::kCtasPerSm : FwdCfg<64, 2>::kCtasPerSm;
+    return hd == 128 ? FwdCfg<128, 1>::kCtasPerSm : FwdCfg<64, 1>::kCtasPerSm;
+}
+
+cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, int grid, cudaStream_t stream) {
+    if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2>(p, grid, stream) : launch_fwd_t<128, 1>(p, grid, stream);
+    return nt == 2 ? launch_fwd_t<64, 2>(p, grid, stream) : launch_fwd_t<64, 1>(p, grid, stream);
+}
+
+cudaError_t launch_combine(const CombineParams& p, int hd, int num_sms, cudaStream_t stream) {
+    const long long rows = (long long)p.B * p.Hq * p.Sq;
+    long long blocks = (rows + 7) / 8;
+    const long long cap = (long long)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    if (hd == 128)
+        gqa_combine_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(p);
+    else
+        gqa_combine_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+unsigned int* device_status_symbol() {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
+    return static_cast<unsigned int*>(ptr);
+}
+
+}  // namespace gqa

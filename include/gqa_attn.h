@@ -1,0 +1,130 @@
+/*
+ * gqa_attn — exact grouped-query attention forward for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libgqa_attn.so.  Plain pointers and sizes only.
+ *
+ * What is computed, for b < B, q-head h < Hq, query position i < Sq:
+ *
+ *   kvh        = h / (Hq / Hk)                  the kv head shared by q-head h's group
+ *   allowed(i) = { j < Sk : !causal  or  j <= i + (Sk - Sq) }
+ *   s_j        = scale * sum_c q[b,i,h,c] * k[b,j,kvh,c]
+ *   out[b,i,h,:] = sum_{j in allowed(i)} exp(s_j) v[b,j,kvh,:] / sum_{j in allowed(i)} exp(s_j)
+ *   lse[b,h,i]   = ln sum_{j in allowed(i)} exp(s_j)
+ *
+ * Sources for the definition:
+ *  - "PyTorch 性能分析深度指南 (第三部分)", section "Attention 的计算挑战":
+ *    Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V.
+ *  - "优化GQA在Flash-Attention中的批量敏感性", section "分组查询注意力的核心设计"
+ *    (and "為什么 GQA 推理吞吐先升后降…4 步速查", section "根因"): Hq must be a multiple
+ *    of Hk; with Hq=6, Hk=2, q-heads 0,1,2 read kv-head 0 and 3,4,5 read kv-head 1.
+ *  - causal=True and softmax_scale = 1/sqrt(d) in every API example of the pages
+ *    ("解锁Stable Diffusion效率瓶颈…", section "动态批量调度"; troubleshooting item
+ *    "精度下降").
+ *  - Readings where the pages are silent: the causal mask is aligned bottom-right
+ *    (identical to top-left when Sq == Sk); lse is the natural log over the scaled
+ *    scores; a row with no allowed key (only possible when causal and Sq > Sk) gets
+ *    out = 0 and lse = -inf.
+ *
+ * Scheduling variants (results do not depend on them beyond fp32 rounding order):
+ *  - pack_gqa: the Hq/Hk query heads of one kv group are folded into the rows of one
+ *    128-row tile, so each K/V tile is read once per group ("优化GQA在Flash-Attention中
+ *    的批量敏感性", section "Flash-Attention的PackGQA优化"; "為什么 GQA 推理吞吐先升后降…",
+ *    section "根因": packing helps when seqlen_q is small or not near a multiple of the
+ *    tile height).
+ *  - num_splits: the key axis is split into num_splits contiguous ranges computed as
+ *    independent partials and merged by an LSE-weighted combine ("為什么 GQA 推理吞吐
+ *    先升后降…", section "修復", table rows for large batch: split the K/V axis, then
+ *    combine).
+ *
+ * Layouts (all row-major, contiguous, device memory owned by the caller):
+ *   q   bf16 [B, Sq, Hq, d]        k, v  bf16 [B, Sk, Hk, d]
+ *   out fp32 [B, Sq, Hq, d]        lse   fp32 [B, Hq, Sq]
+ * d must be 64 or 128.  Every pointer must be 16-byte aligned.
+ *
+ * Threading and ordering: every call is asynchronous on `stream` (a cudaStream_t, or
+ * NULL for the legacy default stream) and never synchronises the host.  Calls may be
+ * made from several host threads.
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GQA_API __attribute__((visibility("default")))
+#else
+#define GQA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_NULL = 1,     /* a required pointer is NULL                              */
+    GQA_ERR_SHAPE = 2,    /* B, Sq, Sk, Hq or Hk < 1, num_splits or pack_gqa invalid, */
+                          /* or a tensor larger than the kernel's 32-bit coordinates  */
+    GQA_ERR_HEADS = 3,    /* Hq is not a multiple of Hk                              */
+    GQA_ERR_HEADDIM = 4,  /* d not in {64, 128}                                      */
+    GQA_ERR_ALIGN = 5,    /* a pointer is not 16-byte aligned                         */
+    GQA_ERR_ARCH = 6,     /* the current device is not sm_100 (B200 class)           */
+    GQA_ERR_ALLOC = 7,    /* split-KV workspace could not be allocated                */
+    GQA_ERR_CUDA = 8,     /* a CUDA runtime/driver call failed (launch, tensor map)   */
+    GQA_ERR_TIMEOUT = 9   /* a bounded in-kernel wait ran out (read back by           */
+                          /* gqa_attn_device_status after the stream has synchronised) */
+} gqa_status;
+
+/*
+ * Forward pass.  Writes out and lse; reads q, k, v.
+ *
+ *   scale       multiplier of q.k (1/sqrt(d) in the pages' examples); any finite value.
+ *   causal      0 or 1.
+ *   pack_gqa    -1 = chosen by gqa_attn_choose, 0 = one q-head per tile, 1 = packed.
+ *   num_splits  0 = chosen by gqa_attn_choose, >= 1 = that many key ranges.  Clamped to
+ *               the number of 128-key blocks and to 16.  With more than one split the
+ *               library allocates stream-ordered scratch (cudaMallocAsync on `stream`,
+ *               freed with cudaFreeAsync after the combine on the same stream) of
+ *               gqa_attn_workspace_bytes(...) bytes.
+ *
+ * Errors: argument errors return before anything is launched or written.  Launch
+ * errors return GQA_ERR_CUDA.  A device-side bounded-wait timeout (which should not
+ * happen) is reported through gqa_attn_device_status.
+ */
+GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out, float* lse,
+                        int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
+                        int pack_gqa, int num_splits, void* stream);
+
+/*
+ * The scheduling heuristic alone (host only, no CUDA call): what gqa_attn_fwd uses when
+ * pack_gqa = -1 / num_splits = 0.  num_sms is the device's SM count (148 on B200; pass
+ * <= 0 for 148).  The pages give four mutually contradictory batch-size tables tuned on
+ * H100 ("解锁Stable Diffusion效率瓶颈…", "动态批量调度" and "三步优化检查清单";
+ * "优化GQA在Flash-Attention中的批量敏感性", strategy 2 and "参数组合"; "為什么 GQA 推理吞吐
+ * 先升后降…", "修復" table); this rule is re-derived for B200 instead: pack when it
+ * computes fewer padded tile rows, split the key axis when the (batch, head, q-tile)
+ * units alone cannot fill the SMs.
+ */
+GQA_API gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
+                           int num_sms, int* pack_gqa, int* num_splits);
+
+/* Bytes of split-KV scratch gqa_attn_fwd allocates for these arguments (0 when
+ * num_splits resolves to 1).  pack_gqa / num_splits follow gqa_attn_fwd's conventions. */
+GQA_API size_t gqa_attn_workspace_bytes(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
+                                int pack_gqa, int num_splits);
+
+/* Static description of a status code. */
+GQA_API const char* gqa_attn_status_string(gqa_status status);
+
+/*
+ * Device-side status word of the current device (GQA_OK or GQA_ERR_TIMEOUT), written by
+ * kernels whose bounded waits ran out.  Synchronous: it waits for the device.  With
+ * reset != 0 the word is cleared after reading.
+ */
+GQA_API gqa_status gqa_attn_device_status(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

@@ -1,0 +1,111 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same
+seeded inputs, element by element, within the stated tolerances."""
+import numpy as np
+import pytest
+
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gqa_exact_attention_b200 as G
+    G.load()
+    yield
+    assert G.gqa_attn_device_status(reset=True) == 0, "an in-kernel wait timed out"
+
+
+def run(q, k, v, causal, pack=-1, splits=0, scale=None):
+    import gqa_exact_attention_b200 as G
+    out, lse = G.gqa_attn_fwd(q, k, v, scale=scale, causal=causal, pack_gqa=pack,
+                              num_splits=splits)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+# --- the tiny configuration: B=1, Hq=6, Hk=2, Sq=Sk=128, d=64, all 8 variants
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("pack", [0, 1])
+@pytest.mark.parametrize("splits", [1, 2])
+def test_tiny_all_variants(causal, pack, splits):
+    seed, shp = 1000, (1, 128, 128, 6, 2, 64)
+    q, k, v = P.device_inputs(seed, *shp)
+    o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(64), causal)
+    out, lse = run(q, k, v, causal, pack, splits)
+    P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"tiny c{causal} p{pack} s{splits}")
+    base, lbase = run(q, k, v, causal, 0, 1)
+    assert (out - base).abs().max().item() <= P.VARIANT_MAX
+    assert (lse - lbase).abs().max().item() <= P.VARIANT_MAX
+
+
+# --- ragged shapes: tails in Sq and Sk, several tiles, head ratios from MHA to MQA
+RAGGED = [
+    # B, Sq, Sk, Hq, Hk, d
+    (2, 77, 300, 8, 2, 128),
+    (1, 300, 300, 4, 4, 128),
+    (2, 130, 257, 8, 1, 64),
+    (1, 1, 700, 32, 8, 128),
+    (3, 5, 129, 6, 3, 64),
+    (1, 384, 200, 4, 2, 128),
+    (1, 200, 384, 8, 4, 64),
+]
+
+
+@pytest.mark.parametrize("shp", RAGGED, ids=[str(s) for s in RAGGED])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("pack,splits", [(0, 1), (1, 1), (0, 3), (1, 2), (-1, 0)])
+def test_ragged(shp, causal, pack, splits):
+    seed = 2000 + sum(shp)
+    q, k, v = P.device_inputs(seed, *shp)
+    o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(shp[-1]), causal)
+    out, lse = run(q, k, v, causal, pack, splits)
+    P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"{shp} c{causal} p{pack} s{splits}")
+
+
+# --- causal with Sq > Sk: leading rows see no key (O = 0, LSE = -inf)
+@pytest.mark.parametrize("pack,splits", [(0, 1), (1, 1), (0, 2), (1, 3)])
+def test_empty_rows(pack, splits):
+    shp = (2, 260, 70, 4, 2, 64)
+    seed = 3000
+    q, k, v = P.device_inputs(seed, *shp)
+    o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(64), 1)
+    assert np.isneginf(l_ref).any()
+    out, lse = run(q, k, v, 1, pack, splits)
+    P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "empty rows")
+    empty = torch.from_numpy(np.isneginf(l_ref)).cuda()
+    assert torch.all(out.permute(0, 2, 1, 3)[empty] == 0)
+
+
+# --- closed forms on the GPU: scale 0 gives the mean of V over the allowed keys;
+#     causal row 0 with Sq == Sk is v_0 exactly.
+def test_scale_zero_and_single_key():
+    shp = (1, 200, 200, 4, 2, 128)
+    seed = 3100
+    q, k, v = P.device_inputs(seed, *shp)
+    out, lse = run(q, k, v, 1, 0, 1, scale=0.0)
+    vf = v.float()
+    csum = torch.cumsum(vf, dim=1) / torch.arange(1, 201, device="cuda").view(1, -1, 1, 1)
+    ref = csum.repeat_interleave(2, dim=2)
+    assert (out - ref).abs().max().item() <= 1e-4
+    ln = torch.log(torch.arange(1, 201, device="cuda", dtype=torch.float32))
+    assert (lse - ln.view(1, 1, -1)).abs().max().item() <= 1e-5
+    out, lse = run(q, k, v, 1, 0, 1)
+    assert torch.equal(out[0, 0, 0], vf[0, 0, 0]) and torch.equal(out[0, 0, 3], vf[0, 0, 1])
+
+
+# --- odd shapes / head ratios: Sq=77 vs Sk=4096 non-causal, d in {64,128},
+#     (Hq,Hk) in {(32,32),(32,8),(32,4),(32,1)}, full oracle
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("hk", [32, 8, 4, 1])
+def test_odd_sq77_sk4096(d, hk):
+    shp = (4, 77, 4096, 32, hk, d)
+    seed = 1004
+    q, k, v = P.device_inputs(seed, *shp)
+    o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(d), 0)
+    out, lse = run(q, k, v, 0)
+    P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"Sq77 d{d} hk{hk}")
