@@ -1,0 +1,449 @@
+#!/usr/bin/env python3
+"""Benchmark of the GQA attention forward on B200.
+
+Default workload: prefill GQA, B=64, Hq=32, Hk=8, Sq=Sk=2048, d=128, bf16 Q/K/V ~ N(0,1)
+(seeded, synthetic), causal, scale 1/sqrt(128), pack_gqa / num_splits from the heuristic.
+One step = one forward over the whole batch.  Rank 0 prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the fp64 CPU oracle (the only reference this project has) on the
+box's host cores, on bounded samples of the same workload.  Other flags (--B, --Sq, ...)
+select another shape for ad-hoc measurement; ``--sweep prefill|decode`` prints one line
+per configuration of the batch-sensitivity sweep or the decode grid.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GQA fwd TFLOPS & tokens/s (Hq32 Hk8 d128 S2K, B16-256); decode HBM GB/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SRC = os.path.join(ROOT, "gqa_exact_attention_b200", "csrc", "fwd_sm100.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- work accounting
+
+def causal_pairs(Sq, Sk):
+    """Number of (query, key) pairs the causal mask allows (bottom-right aligned)."""
+    tot = 0
+    off = Sk - Sq
+    # row i allows min(Sk, max(0, i + 1 + off)) keys
+    lo = max(0, -off)  # first row with at least one key
+    full_from = max(lo, Sk - off - 1)  # rows from here see all Sk keys
+    full_from = min(max(full_from, lo), Sq)
+    # rows lo .. full_from-1: i + 1 + off keys
+    n = full_from - lo
+    if n > 0:
+        a = lo + 1 + off
+        tot += n * a + n * (n - 1) // 2
+    tot += (Sq - full_from) * Sk
+    return tot
+
+
+def flops(B, Sq, Sk, Hq, d, causal):
+    """4 B Hq Sq Sk d for non-causal; the allowed pairs (Sq Sk / 2 when Sq = Sk, up to
+    the diagonal term) for causal: 2 flops per multiply-add in QK^T and in PV."""
+    pairs = causal_pairs(Sq, Sk) if causal else Sq * Sk
+    if causal and Sq == Sk:
+        pairs = Sq * Sk / 2  # the pages' convention: halved for causal
+    return 4.0 * B * Hq * d * pairs
+
+
+def hbm_bytes(B, Sq, Sk, Hq, Hk, d):
+    """Algorithmic bytes: read Q, K, V once (bf16), write O (fp32) and LSE (fp32)."""
+    return 2 * B * Sq * Hq * d + 2 * 2 * B * Sk * Hk * d + 4 * B * Sq * Hq * d + 4 * B * Hq * Sq
+
+
+# ----------------------------------------------------------------- environment
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_hash():
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(workload_key):
+    """DRAM bytes per launch from a committed ncu capture, if it was taken on the current
+    kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    if t.get("kernel_sha256_16") != kernel_hash():
+        return None
+    e = t.get("workloads", {}).get(workload_key)
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, mx, util = float(parts[1]), float(parts[2]), float(parts[4])
+            except ValueError:
+                continue
+            smax = mx
+            if util >= 50:
+                sm.append(clk)
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples_under_load": len(sm)}
+
+
+# ----------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local, pg
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, x):
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(cfg, budget_s):
+    """Time the fp64 oracle on whole batch elements of the workload until about
+    budget_s seconds of CPU work; returns (flops/s, threads, description)."""
+    import inputs
+    import oracle
+    B, Sq, Sk, Hq, Hk, d, causal = (cfg[k] for k in ("B", "Sq", "Sk", "Hq", "Hk", "d", "causal"))
+    scale = 1.0 / math.sqrt(d)
+
+    def one(nb, seed_off):
+        # nb batch elements, all heads (regenerated from the same seeded definition)
+        qs, ks = (nb, Sq, Hq, d), (nb, Sk, Hk, d)
+        f = inputs.bf16_bits_to_f64
+        q = f(inputs.bits_range(cfg["seed"], inputs.TID_Q, seed_off * Sq * Hq * d, nb * Sq * Hq * d)).reshape(qs)
+        k = f(inputs.bits_range(cfg["seed"], inputs.TID_K, seed_off * Sk * Hk * d, nb * Sk * Hk * d)).reshape(ks)
+        v = f(inputs.bits_range(cfg["seed"], inputs.TID_V, seed_off * Sk * Hk * d, nb * Sk * Hk * d)).reshape(ks)
+        t0 = time.perf_counter()
+        _, _, threads = oracle.attn_fwd(q, k, v, scale, causal, return_threads=True)
+        return time.perf_counter() - t0, threads
+
+    # calibrate on one sequence restricted to a few heads' worth of time
+    t1, threads = one(1, 0)
+    nb = max(1, min(B, int(budget_s / max(t1, 1e-3))))
+    if nb > 1:
+        tn, threads = one(nb, 1)
+        total_t, total_b = t1 + tn, 1 + nb
+    else:
+        total_t, total_b = t1, 1
+    rate = flops(total_b, Sq, Sk, Hq, d, causal) / total_t
+    desc = (f"{total_b} of {B} sequences (all {Hq} heads, Sq={Sq}, Sk={Sk}), fp64 oracle, "
+            f"{total_t:.1f} s")
+    return rate, threads, desc
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_gpu(args, cfg):
+    import torch
+
+    import gqa_exact_attention_b200 as G
+    import inputs  # seeded input generator (no attention arithmetic)
+
+    rank, world, local, pg = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    G.load()
+    B, Sq, Sk, Hq, Hk, d, causal = (cfg[k] for k in ("B", "Sq", "Sk", "Hq", "Hk", "d", "causal"))
+    pack, splits = G.gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, causal) if (args.pack < 0 and args.splits <= 0) \
+        else (args.pack, args.splits)
+    if args.pack >= 0:
+        pack = args.pack
+    if args.splits > 0:
+        splits = args.splits
+    seed = cfg["seed"] + rank
+    q = inputs.device_tensor(seed, inputs.TID_Q, (B, Sq, Hq, d), device=dev)
+    k = inputs.device_tensor(seed, inputs.TID_K, (B, Sk, Hk, d), device=dev)
+    v = inputs.device_tensor(seed, inputs.TID_V, (B, Sk, Hk, d), device=dev)
+    out = torch.empty((B, Sq, Hq, d), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 + (1 if splits > 1 else 0)
+
+    def step():
+        G.gqa_attn_fwd(q, k, v, out=out, lse=lse, causal=causal, pack_gqa=pack,
+                       num_splits=splits, stream=stream)
+
+    sampler = ClockSampler(local if world > 1 else 0) if rank == 0 or world > 1 else None
+    if sampler:
+        sampler.start()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: K steps, events per launch on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(pg)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg)
+    total_ms = max_over_ranks(pg, t_start.elapsed_time(t_end))
+    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    launch_ms = max_over_ranks(pg, launch_ms)
+    ms_per_step = total_ms / args.steps
+    if G.gqa_attn_device_status(reset=True) != 0:
+        raise SystemExit("an in-kernel bounded wait timed out during the benchmark")
+
+    # ---- end to end through the public API: pinned host inputs in, results out
+    q_h = q.cpu().pin_memory()
+    k_h = k.cpu().pin_memory()
+    v_h = v.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(1, min(args.steps, 20))
+    barrier(pg)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg)
+    e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1)) / e_steps
+    clocks = sampler.stop() if sampler else None
+
+    fl = flops(B, Sq, Sk, Hq, d, causal)
+    by = hbm_bytes(B, Sq, Sk, Hq, Hk, d)
+    peaks, peak_src = load_peaks()
+    decode_like = Sq * (Hq // Hk) <= 128 and not causal
+    timed_s = total_ms / 1e3
+    if decode_like:
+        achieved = by / (launch_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+        value = world * by / (ms_per_step / 1e3) / 1e9
+        unit = "GB/s"
+        e2e_value = world * by / (e2e_ms / 1e3) / 1e9
+    else:
+        pk_key = "bf16_tflops_sustained" if timed_s > 1.0 else "bf16_tflops"
+        achieved = fl / (launch_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[pk_key], "unit": "TFLOP/s",
+                "frac": achieved / peaks[pk_key]}
+        value = world * fl / (ms_per_step / 1e3) / 1e12
+        unit = "TFLOP/s"
+        e2e_value = world * fl / (e2e_ms / 1e3) / 1e12
+    roof["peak_source"] = f"{peak_src}:" + ("hbm_gbs" if decode_like else pk_key)
+    roof["traffic"] = traffic_for(cfg["name"])
+    roof["kernel"] = "gqa_fwd_kernel"
+
+    tokens = B * (Sq if Sq > 1 else 1)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) rounded to bf16)",
+        "config": {"workload": cfg["name"], "B": B, "Sq": Sq, "Sk": Sk, "Hq": Hq, "Hk": Hk,
+                   "d": d, "causal": bool(causal), "pack_gqa": pack, "num_splits": splits,
+                   "out_dtype": "fp32", "l2": cfg["l2"],
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "tokens_per_s": round(world * tokens / (ms_per_step / 1e3), 1),
+        "tflops": round(world * fl / (ms_per_step / 1e3) / 1e12, 3),
+        "hbm_gbs": round(world * by / (ms_per_step / 1e3) / 1e9, 1),
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, threads, desc = oracle_sample(cfg, args.cpu_budget)
+        if decode_like:
+            cv = by / (fl / rate) / 1e9
+        else:
+            cv = rate / 1e12
+        line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": threads, "kind": "oracle",
+                                "sample": desc}
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, cfg):
+    """The fp64 oracle as it stands, on host cores, bounded samples of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    B, Sq, Sk, Hq, Hk, d, causal = (cfg[k] for k in ("B", "Sq", "Sk", "Hq", "Hk", "d", "causal"))
+    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, budget / 4)
+    rates, threads, desc = [], 1, ""
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r, threads, desc = oracle_sample(cfg, budget)
+        rates.append(r)
+    wall = time.perf_counter() - t0
+    fl = flops(B, Sq, Sk, Hq, d, causal)
+    by = hbm_bytes(B, Sq, Sk, Hq, Hk, d)
+    rate = statistics.mean(rates)
+    decode_like = Sq * (Hq // Hk) <= 128 and not causal
+    value, unit = ((by / (fl / rate) / 1e9, "GB/s") if decode_like else (rate / 1e12, "TFLOP/s"))
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": unit,
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * wall / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) rounded to bf16)",
+        "config": {"workload": cfg["name"], "B": B, "Sq": Sq, "Sk": Sk, "Hq": Hq, "Hk": Hk,
+                   "d": d, "causal": bool(causal), "out_dtype": "fp64", "l2": cfg["l2"]},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--B", type=int, default=64)
+    ap.add_argument("--Sq", type=int, default=2048)
+    ap.add_argument("--Sk", type=int, default=2048)
+    ap.add_argument("--Hq", type=int, default=32)
+    ap.add_argument("--Hk", type=int, default=8)
+    ap.add_argument("--d", type=int, default=128)
+    ap.add_argument("--causal", type=int, default=1)
+    ap.add_argument("--pack", type=int, default=-1)
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    default = (args.B, args.Sq, args.Sk, args.Hq, args.Hk, args.d, args.causal) == (64, 2048, 2048, 32, 8, 128, 1)
+    name = ("prefill B=64 Hq=32 Hk=8 Sq=Sk=2048 d=128 causal" if default else
+            f"B={args.B} Hq={args.Hq} Hk={args.Hk} Sq={args.Sq} Sk={args.Sk} d={args.d} "
+            f"{'causal' if args.causal else 'non-causal'}")
+    in_bytes = 2 * (args.B * args.Sq * args.Hq * args.d + 2 * args.B * args.Sk * args.Hk * args.d)
+    cfg = {"name": name, "B": args.B, "Sq": args.Sq, "Sk": args.Sk, "Hq": args.Hq, "Hk": args.Hk,
+           "d": args.d, "causal": args.causal, "seed": 1001,
+           "l2": (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step)"
+                  if in_bytes > 126e6 else f"inputs {in_bytes / 1e6:.1f} MB, L2-resident")}
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_gpu(args, cfg)
+
+
+if __name__ == "__main__":
+    main()
