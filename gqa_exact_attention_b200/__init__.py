@@ -15,7 +15,8 @@ import os
 
 __all__ = [
     "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes", "gqa_attn_status_string",
-    "gqa_attn_device_status", "GqaError", "lib_path", "load",
+    "gqa_attn_device_status", "gqa_attn_fwd_noalloc", "GqaError", "lib_path", "load",
+    "GQA_NOALLOC_SCRATCH_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -25,8 +26,12 @@ GQA_OK = 0
 STATUS_NAMES = {
     0: "GQA_OK", 1: "GQA_ERR_NULL", 2: "GQA_ERR_SHAPE", 3: "GQA_ERR_HEADS",
     4: "GQA_ERR_HEADDIM", 5: "GQA_ERR_ALIGN", 6: "GQA_ERR_ARCH", 7: "GQA_ERR_ALLOC",
-    8: "GQA_ERR_CUDA", 9: "GQA_ERR_TIMEOUT",
+    8: "GQA_ERR_CUDA", 9: "GQA_ERR_TIMEOUT", 10: "GQA_ERR_SCRATCH",
 }
+
+# size of the library's fixed split-KV scratch used by gqa_attn_fwd_noalloc (the header's
+# GQA_NOALLOC_SCRATCH_BYTES)
+GQA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class GqaError(RuntimeError):
@@ -65,6 +70,8 @@ def load():
     L.gqa_attn_status_string.restype = ctypes.c_char_p
     L.gqa_attn_device_status.argtypes = [i]
     L.gqa_attn_device_status.restype = i
+    L.gqa_attn_fwd_noalloc.argtypes = [p, p, p, p, p, i, i, i, i, i, i, f, i, i, i, p]
+    L.gqa_attn_fwd_noalloc.restype = i
     _lib = L
     return L
 
@@ -102,7 +109,7 @@ def gqa_attn_device_status(reset: bool = False) -> int:
 
 
 def gqa_attn_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, pack_gqa=-1,
-                 num_splits=0, stream=None):
+                 num_splits=0, stream=None, _entry="gqa_attn_fwd"):
     """out, lse = gqa_attn_fwd(q, k, v, ...) on the current CUDA stream.
 
     q: bf16 [B, Sq, Hq, d]; k, v: bf16 [B, Sk, Hk, d]; all contiguous CUDA tensors.
@@ -132,8 +139,22 @@ def gqa_attn_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, pack_gqa
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
-        _check(load().gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                   lse.data_ptr(), B, Sq, Sk, Hq, Hk, d, float(scale),
-                                   int(bool(causal)), int(pack_gqa), int(num_splits),
-                                   stream.cuda_stream))
+        _check(getattr(load(), _entry)(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       out.data_ptr(), lse.data_ptr(), B, Sq, Sk, Hq, Hk, d,
+                                       float(scale), int(bool(causal)), int(pack_gqa),
+                                       int(num_splits), stream.cuda_stream))
     return out, lse
+
+
+def gqa_attn_fwd_noalloc(q, k, v, out, lse, scale=None, causal=False, pack_gqa=-1,
+                         num_splits=0, stream=None):
+    """gqa_attn_fwd for callers that must not allocate device memory (a serving process
+    that reserved its device memory up front, code that must not block on the device,
+    a host under another runtime's allocator).  ``out`` and ``lse`` are required; the
+    split-KV partials use the library's fixed scratch of GQA_NOALLOC_SCRATCH_BYTES per
+    device, and calls that overlap on the GPU race on it."""
+    if out is None or lse is None:
+        raise ValueError("gqa_attn_fwd_noalloc writes into caller-provided out and lse")
+    return gqa_attn_fwd(q, k, v, out=out, lse=lse, scale=scale, causal=causal,
+                        pack_gqa=pack_gqa, num_splits=num_splits, stream=stream,
+                        _entry="gqa_attn_fwd_noalloc")

@@ -196,6 +196,7 @@ const char* gqa_attn_status_string(gqa_status s) {
         case GQA_ERR_ALLOC: return "split-KV workspace allocation failed";
         case GQA_ERR_CUDA: return "CUDA call failed";
         case GQA_ERR_TIMEOUT: return "an in-kernel bounded wait timed out";
+        case GQA_ERR_SCRATCH: return "split-KV partials exceed the library's static scratch";
     }
     return "unknown status";
 }
@@ -316,3 +317,80 @@ gqa_status gqa_attn_device_status(int reset) {
 }
 
 }  // extern "C"
+
+namespace gqa {
+
+// Forward with caller-provided split-KV scratch (no allocation): used by
+// gqa_attn_fwd_noalloc.  Same validation and plan as gqa_attn_fwd.
+gqa_status fwd_with_scratch(const void* q, const void* k, const void* v, float* out, float* lse,
+                            int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
+                            int pack_gqa, int num_splits, void* stream_ptr, void* scratch,
+                            size_t scratch_bytes) {
+    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
+    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
+    if (st != GQA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+        return GQA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return GQA_ERR_SHAPE;
+    int dev = 0;
+    DeviceInfo info;
+    st = device_info(&dev, &info);
+    if (st != GQA_OK) return st;
+    if (!info.ok) return GQA_ERR_ARCH;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+
+    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms);
+    const int g = Hq / Hk;
+    const size_t rows = (size_t)B * Hq * Sq;
+    const size_t need = pl.splits > 1 ? (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float) : 0;
+    if (need > 0 && (scratch == nullptr || need > scratch_bytes)) return GQA_ERR_SCRATCH;
+
+    FwdParams p{};
+    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM) ||
+        !encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
+        !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
+        return GQA_ERR_CUDA;
+    p.out = out;
+    p.lse = lse;
+    p.B = B;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.Hq = Hq;
+    p.Hk = Hk;
+    p.g = g;
+    p.pack = pl.pack;
+    p.pos_per_tile = pl.pos_per_tile;
+    p.rows_valid = pl.rows_valid;
+    p.causal = causal ? 1 : 0;
+    p.num_splits = pl.splits;
+    p.n_hg = pl.n_hg;
+    p.n_mt = pl.n_mt;
+    p.n_units = (int)pl.units;
+    p.kv_blocks = pl.kv_blocks;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.div_g = make_fastdiv((uint32_t)g);
+    p.status = nullptr;
+    p.timeout_ns = timeout_ns();
+    if (pl.splits > 1) {
+        p.o_part = static_cast<float*>(scratch);
+        p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
+    }
+    const int slots = info.sms * fwd_ctas_per_sm(d, pl.nt);
+    const int grid = (int)(pl.units < slots ? pl.units : slots);
+    if (launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) return GQA_ERR_CUDA;
+    if (pl.splits > 1) {
+        CombineParams c{};
+        c.o_part = p.o_part;
+        c.lse_part = p.lse_part;
+        c.out = out;
+        c.lse = lse;
+        c.B = B;
+        c.Sq = Sq;
+        c.Hq = Hq;
+        c.num_splits = pl.splits;
+        if (launch_combine(c, d, info.sms, stream) != cudaSuccess) return GQA_ERR_CUDA;
+    }
+    return GQA_OK;
+}
+
+}  // namespace gqa

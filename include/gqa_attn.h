@@ -71,8 +71,10 @@ typedef enum {
     GQA_ERR_ARCH = 6,     /* the current device is not sm_100 (B200 class)           */
     GQA_ERR_ALLOC = 7,    /* split-KV workspace could not be allocated                */
     GQA_ERR_CUDA = 8,     /* a CUDA runtime/driver call failed (launch, tensor map)   */
-    GQA_ERR_TIMEOUT = 9   /* a bounded in-kernel wait ran out (read back by           */
+    GQA_ERR_TIMEOUT = 9,  /* a bounded in-kernel wait ran out (read back by           */
                           /* gqa_attn_device_status after the stream has synchronised) */
+    GQA_ERR_SCRATCH = 10  /* gqa_attn_fwd_noalloc: the split-KV partials do not fit the */
+                          /* library's static scratch (GQA_NOALLOC_SCRATCH_BYTES)       */
 } gqa_status;
 
 /*
@@ -122,6 +124,44 @@ GQA_API const char* gqa_attn_status_string(gqa_status status);
  * reset != 0 the word is cleared after reading.
  */
 GQA_API gqa_status gqa_attn_device_status(int reset);
+
+/*
+ * gqa_attn_fwd_noalloc — the same forward as gqa_attn_fwd, with the same arguments and
+ * results, for callers that must not allocate device memory.  (The pages have no
+ * counterpart; this is an interface addition of this library.)
+ *
+ * Who needs it: a serving process that reserves nearly all device memory up front
+ * (weights, KV-cache pools) and forbids any allocation on its hot path, so an
+ * allocation there can fail mid-step with nothing to fall back on; code that must not
+ * make a call that may block on the device, as cudaMalloc/cudaFree can; and hosts
+ * that embed this library under another runtime's allocator, which owns device memory
+ * and does not expect a library to grab some of it behind its back.  gqa_attn_fwd
+ * allocates the split-KV partials with cudaMallocAsync when num_splits > 1; this entry
+ * point never allocates.
+ *
+ * Scratch: the split-KV partials (O_s and lse_s per split) live in one fixed array
+ * inside the library, GQA_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads the
+ * library, held until the process exits.  A call whose partials need more, i.e.
+ * num_splits * B * Hq * Sq * (d + 1) * 4 bytes after num_splits is resolved, returns
+ * GQA_ERR_SCRATCH before anything is launched.  With num_splits resolving to 1 no
+ * scratch is used.
+ *
+ * The array is shared by every call on a device and keeps the last call's contents.
+ * Nothing in it has to start at zero: every partial element is written before the
+ * combine reads it.  Calls whose kernels overlap on the GPU (different streams, or
+ * different host threads without ordering between them) race on the array; order them
+ * on one stream or with events.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current.  Make that first call before any
+ * stream capture on the device.  A failed look-up returns GQA_ERR_CUDA.
+ */
+#define GQA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+GQA_API gqa_status gqa_attn_fwd_noalloc(const void* q, const void* k, const void* v, float* out,
+                                        float* lse, int B, int Sq, int Sk, int Hq, int Hk, int d,
+                                        float scale, int causal, int pack_gqa, int num_splits,
+                                        void* stream);
 
 #ifdef __cplusplus
 }

@@ -21,7 +21,7 @@ def declared_symbols():
 def test_header_declares_the_entry_points():
     assert declared_symbols() == sorted([
         "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes",
-        "gqa_attn_status_string", "gqa_attn_device_status"])
+        "gqa_attn_status_string", "gqa_attn_device_status", "gqa_attn_fwd_noalloc"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -79,7 +79,7 @@ def test_pages_head_constraint_example():
 
 
 def test_status_strings():
-    for c in range(10):
+    for c in range(11):
         assert G.gqa_attn_status_string(c) != "unknown status"
     assert G.gqa_attn_status_string(42) == "unknown status"
 
