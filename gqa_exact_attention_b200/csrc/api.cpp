@@ -79,14 +79,23 @@ Plan make_plan(int B, int Sq, int Sk, int Hq, int Hk, int pack) {
     return pl;
 }
 
+// Split count minimising the modelled time: waves(s) x (key blocks per split + a fixed
+// per-unit cost of about one block: Q load, pipeline fill, epilogue).  A persistent CTA
+// per SM takes units in a static stride, so a partial last wave costs a whole unit time.
 int choose_splits(const Plan& pl, int d, int num_sms) {
-    const int slots = num_sms * gqa::fwd_ctas_per_sm(d, pl.nt);
-    if (pl.units >= slots) return 1;
-    int s = ceil_div(slots, pl.units);
-    const int cap = pl.kv_blocks / 2 > 1 ? pl.kv_blocks / 2 : 1;
-    if (s > cap) s = cap;
-    if (s > kMaxSplits) s = kMaxSplits;
-    return s < 1 ? 1 : s;
+    const long long slots = (long long)num_sms * gqa::fwd_ctas_per_sm(d, pl.nt);
+    const int smax = pl.kv_blocks < kMaxSplits ? pl.kv_blocks : kMaxSplits;
+    int best = 1;
+    double best_t = 0.0;
+    for (int s = 1; s <= smax; ++s) {
+        const long long waves = (pl.units * s + slots - 1) / slots;
+        const double t = (double)waves * ((double)pl.kv_blocks / s + 1.0);
+        if (s == 1 || t < best_t * 0.97) {  // a split must buy at least 3 %
+            best = s;
+            best_t = t;
+        }
+    }
+    return best;
 }
 
 int clamp_splits(int s, int kv_blocks) {
@@ -169,6 +178,15 @@ gqa_status device_info(int* dev_out, DeviceInfo* info) {
     if (dev >= 0 && dev < 64) cache[dev] = di;
     *info = di;
     return GQA_OK;
+}
+
+// Batches per scheduling window: as many as keep the window's K and V within ~48 MB of
+// the 126 MB L2 (the rest holds Q tiles and output lines in flight).
+int batch_window(int B, int Sk, int Hk, int d) {
+    const double kv_per_batch = 4.0 * Sk * Hk * d;  // K and V, bf16
+    int w = (int)(48.0e6 / (kv_per_batch > 1.0 ? kv_per_batch : 1.0));
+    if (w < 1) w = 1;
+    return w < B ? w : B;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -261,6 +279,7 @@ gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out,
     p.n_hg = pl.n_hg;
     p.n_mt = pl.n_mt;
     p.n_units = (int)pl.units;
+    p.batch_window = batch_window(B, Sk, Hk, d);
     p.kv_blocks = pl.kv_blocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.div_g = gqa::make_fastdiv((uint32_t)g);
@@ -366,6 +385,7 @@ gqa_status fwd_with_scratch(const void* q, const void* k, const void* v, float* 
     p.n_hg = pl.n_hg;
     p.n_mt = pl.n_mt;
     p.n_units = (int)pl.units;
+    p.batch_window = batch_window(B, Sk, Hk, d);
     p.kv_blocks = pl.kv_blocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.div_g = make_fastdiv((uint32_t)g);

@@ -34,6 +34,7 @@ struct FwdParams {
     int n_hg;          // heads-or-groups per batch: Hq (unpacked) or Hk (packed)
     int n_mt;          // CTA-units along the query axis per (b, hg)
     int n_units;       // n_mt * B * n_hg * num_splits
+    int batch_window;  // batches per scheduling window (their K/V fits in L2)
     int kv_blocks;     // ceil(Sk / 128)
     float scale_log2;  // scale * log2(e)
     FastDiv div_g;     // row -> (position, head-in-group) for packed tiles

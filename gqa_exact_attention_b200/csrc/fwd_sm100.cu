@@ -40,19 +40,43 @@ struct FwdCfg {
     static constexpr int kChunks = HD / 64;              // 128-byte column chunks of a row
     static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kSlots = (NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 2 : 4);
-    static constexpr int kSoftmaxWarps = 4 * NT;
-    static constexpr int kThreads = (2 + kSoftmaxWarps) * 32;
-    static constexpr int kCtasPerSm = (NT == 2) ? 1 : 2;
+    static constexpr int kSlots = (NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 5 : 10);
+    // warpgroups: 0 = TMA producer + MMA issuer, 1..NT = softmax (one per tile),
+    // NT+1 = epilogue
+    static constexpr int kWarpgroups = 2 + NT;
+    static constexpr int kThreads = kWarpgroups * 128;
+    static constexpr int kCtasPerSm = 1;
+    // registers: at launch (65536 / threads, rounded down to 8), then redistributed with
+    // setmaxnreg; the per-thread sum over the warpgroups equals warpgroups x launch regs,
+    // so every increase is covered by the decreases (each sub-partition holds one warp of
+    // each warpgroup)
+    static constexpr int kLaunchRegs = ((65536 / kThreads) / 8) * 8;
+    static constexpr int kRegsLoad = NT == 2 ? 96 : 56;
+    static constexpr int kRegsSoftmax = NT == 2 ? 168 : 232;
+    static constexpr int kRegsEpilogue = kWarpgroups * kLaunchRegs - kRegsLoad - NT * kRegsSoftmax;
+    static_assert(kRegsLoad + NT * kRegsSoftmax + kRegsEpilogue == kWarpgroups * kLaunchRegs,
+                  "register split must add up to the launch allocation");
+    static_assert(kRegsEpilogue >= 64 && kRegsEpilogue % 8 == 0, "epilogue registers");
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
-    static constexpr int kNumBars = 2 * kSlots + 6 * NT + 1;
-    static constexpr int kSmemBytes =
-        1024 /* alignment slack */ + NT * kTileBytes + kSlots * kTileBytes + 8 * kNumBars + 16;
+    static constexpr int kNumBars = 2 * kSlots + 7 * NT + 1;
+    static constexpr int kStatsBytes = 2 * NT * 2 * 128 * 4;  // (m, l) per row, 2 buffers
+    static constexpr int kSmemBytes = 1024 /* alignment slack */ + NT * kTileBytes +
+                                      kSlots * kTileBytes + 8 * kNumBars + kStatsBytes + 16;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, HD, true);
     __host__ __device__ static constexpr int s_col(int t) { return t * 128; }
     __host__ __device__ static constexpr int o_col(int t) { return NT * 128 + t * HD; }
 };
+
+template <uint32_t R>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
 
 // Geometry of one work unit, computed identically by every role.
 template <int NT>
@@ -64,16 +88,25 @@ struct UnitGeom {
     int nblk;       // max over tiles of n[t]
 };
 
+// Unit order: batches are taken in windows of p.batch_window (sized on the host so a
+// window's K/V fits in L2); inside a window the query tiles go latest first (the
+// heaviest under a causal mask), then batch, then head-or-group, then split.  With a
+// static stride over the persistent CTAs this spreads heavy and light tiles evenly and
+// keeps every K/V block's readers close together in time.
 template <int NT>
 __device__ __forceinline__ UnitGeom<NT> unit_geom(int u, const FwdParams& p) {
     UnitGeom<NT> g;
-    g.split = u % p.num_splits;
-    u /= p.num_splits;
-    g.hg = u % p.n_hg;
-    u /= p.n_hg;
-    g.b = u % p.B;
-    u /= p.B;
-    const int mt = p.n_mt - 1 - u;  // longest (latest-position) units first
+    const int per_batch = p.n_hg * p.n_mt * p.num_splits;
+    const int w = u / (p.batch_window * per_batch);
+    int r = u - w * p.batch_window * per_batch;
+    const int b0 = w * p.batch_window;
+    const int nb = min(p.batch_window, p.B - b0);
+    g.split = r % p.num_splits;
+    r /= p.num_splits;
+    g.hg = r % p.n_hg;
+    r /= p.n_hg;
+    g.b = b0 + r % nb;
+    const int mt = p.n_mt - 1 - r / nb;
     g.kvh = p.pack ? g.hg : g.hg / p.g;
     int kb_end[NT];
     int kb_union = 0;
@@ -109,6 +142,28 @@ __device__ __forceinline__ int pick(const int (&a)[NT], int t) {
     return v;
 }
 
+// Row r of tile t of a unit -> (query position, q-head); row_ok when it maps to a real
+// output row.  PackGQA: r = position_in_tile * g + head_in_group.
+struct RowMap {
+    int pos, head;
+    bool ok;
+};
+__device__ __forceinline__ RowMap row_map(const FwdParams& p, int pos0, int hg, int row) {
+    RowMap m;
+    if (p.pack) {
+        uint32_t pr, hh;
+        fastdivmod((uint32_t)row, p.div_g, pr, hh);
+        m.pos = pos0 + (int)pr;
+        m.head = hg * p.g + (int)hh;
+        m.ok = row < p.rows_valid && m.pos < p.Sq;
+    } else {
+        m.pos = pos0 + row;
+        m.head = hg;
+        m.ok = m.pos < p.Sq;
+    }
+    return m;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting or when
 // this wait ran past the time limit (then it records the timeout and starts the abort).
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
@@ -139,7 +194,7 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const 
 }
 
 template <int HD, int NT>
-__global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCtasPerSm)
+__global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
     gqa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<HD, NT>;
     extern __shared__ uint8_t smem_raw[];
@@ -150,7 +205,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
     const uint32_t sQ = base;
     const uint32_t sKV = base + NT * C::kTileBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NT * C::kTileBytes + C::kSlots * C::kTileBytes);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+    float* stats = reinterpret_cast<float*>(bars + C::kNumBars);  // [2][NT][2][128]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stats + 2 * NT * 2 * 128);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const uint32_t bar0 = smem_u32(bars);
@@ -162,10 +218,12 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
     auto p_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 3 * NT + t); };
     auto o_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 4 * NT + t); };
     auto o_empty = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 5 * NT + t); };
-    const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 6 * NT);
+    auto st_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 6 * NT + t); };
+    const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 7 * NT);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kSlots; ++s) {
@@ -179,6 +237,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
             mbar_init(p_full(t), 128);
             mbar_init(o_full(t), 1);
             mbar_init(o_empty(t), 128);
+            mbar_init(st_full(t), 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0u;
@@ -198,189 +257,197 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
-            uint32_t qn[NT] = {};  // Q loads issued per tile
-            bool ok = true;
-            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                const UnitGeom<NT> g = unit_geom<NT>(u, p);
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (g.n[t] == 0 || !ok) continue;
-                    if (qn[t] > 0) ok = wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p);
-                    if (!ok) break;
-                    const int rows = p.pack ? p.rows_valid : kBlockM;
-                    mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
-                    const int hcoord = p.pack ? g.hg * p.g : g.hg;
-#pragma unroll
-                    for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q, q_full(t),
-                                    c * 64, hcoord, g.pos0[t], g.b);
-                    ++qn[t];
-                }
-                for (int it = 0; it < g.nblk && ok; ++it) {
-                    const int kpos = (g.kb_lo + it) * kBlockN;
-#pragma unroll
-                    for (int w = 0; w < 2; ++w) {
-                        const int slot = ld % C::kSlots;
-                        if (ld >= (uint32_t)C::kSlots)
-                            ok = wait_bounded(kv_empty(slot), ((ld / C::kSlots) - 1) & 1u, abort_flag, p);
-                        if (!ok) break;
-                        mbar_arrive_expect_tx(kv_full(slot), (uint32_t)C::kTileBytes);
-#pragma unroll
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes,
-                                        w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v,
-                                        kv_full(slot), c * 64, g.kvh, kpos, g.b);
-                        ++ld;
-                    }
-                }
-            }
-            if (!ok) {
-                // let the copies already issued land before the CTA's memory is released
-                const uint32_t first = ld > (uint32_t)C::kSlots ? ld - C::kSlots : 0u;
-                for (uint32_t l = first; l < ld; ++l)
-                    wait_drain(kv_full(l % C::kSlots), (l / C::kSlots) & 1u, p);
-                for (int t = 0; t < NT; ++t)
-                    if (qn[t] > 0) wait_drain(q_full(t), (qn[t] - 1) & 1u, p);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t ld = 0;
-            uint32_t qn[NT] = {}, pn[NT] = {}, on[NT] = {};
-            bool ok = true;
-
-            auto issue_s = [&](int t, int slot) {
-                const uint32_t a0 = sQ + t * C::kTileBytes;
-                const uint32_t b0 = sKV + slot * C::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    mma_ss(tmem + C::s_col(t), sdesc_sw128(a0 + off, 16, 1024),
-                           sdesc_sw128(b0 + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
-                }
-            };
-            auto issue_pv = [&](int t, int slot, bool accumulate) {
-                const uint32_t b0 = sKV + slot * C::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk)
-                    mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
-                           sdesc_sw128(b0 + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
-                           (accumulate || kk > 0) ? 1u : 0u);
-            };
-
-            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                const UnitGeom<NT> g = unit_geom<NT>(u, p);
-                if (g.nblk == 0) continue;
-                // first key block: S_t for every tile that has keys
-                int slot_k = ld % C::kSlots;
-                ok = wait_bounded(kv_full(slot_k), (ld / C::kSlots) & 1u, abort_flag, p);
-                if (!ok) break;
-                ++ld;
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (g.n[t] == 0 || !ok) continue;
-                    ok = wait_bounded(q_full(t), qn[t] & 1u, abort_flag, p);
-                    if (!ok) break;
-                    ++qn[t];
-                    tc_fence_after();
-                    issue_s(t, slot_k);
-                    mma_commit(s_full(t));
-                    if (g.n[t] == 1) mma_commit(q_empty(t));
-                }
-                if (!ok) break;
-                mma_commit(kv_empty(slot_k));
-
-                for (int it = 0; it < g.nblk && ok; ++it) {
-                    const int slot_v = ld % C::kSlots;
-                    ok = wait_bounded(kv_full(slot_v), (ld / C::kSlots) & 1u, abort_flag, p);
-                    if (!ok) break;
-                    ++ld;
-                    // K of the next block: waited for only when its first S is issued
-                    const bool next = it + 1 < g.nblk;
-                    const uint32_t ld_n = ld;
-                    const int slot_n = ld_n % C::kSlots;
-                    bool k_ready = false;
-                    if (next) ++ld;
-                    tc_fence_after();
+    if (wg == 0) {
+        regs_dec<C::kRegsLoad>();
+        if (warp == 0) {
+            // -------------------------------------------------------- TMA producer
+            if (lane == 0) {
+                uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
+                uint32_t qn[NT] = {};  // Q loads issued per tile
+                bool ok = true;
+                for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                    const UnitGeom<NT> g = unit_geom<NT>(u, p);
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
-                        if (it >= g.n[t] || !ok) continue;
-                        ok = wait_bounded(p_full(t), pn[t] & 1u, abort_flag, p);
+                        if (g.n[t] == 0 || !ok) continue;
+                        if (qn[t] > 0) ok = wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p);
                         if (!ok) break;
-                        ++pn[t];
-                        if (it == 0 && on[t] > 0) {
-                            // the previous unit's epilogue must have read O_t out
-                            ok = wait_bounded(o_empty(t), (on[t] - 1) & 1u, abort_flag, p);
+                        const int rows = p.pack ? p.rows_valid : kBlockM;
+                        mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
+                        const int hcoord = p.pack ? g.hg * p.g : g.hg;
+#pragma unroll
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
+                                        q_full(t), c * 64, hcoord, g.pos0[t], g.b);
+                        ++qn[t];
+                    }
+                    for (int it = 0; it < g.nblk && ok; ++it) {
+                        const int kpos = (g.kb_lo + it) * kBlockN;
+#pragma unroll
+                        for (int w = 0; w < 2; ++w) {
+                            const int slot = ld % C::kSlots;
+                            if (ld >= (uint32_t)C::kSlots)
+                                ok = wait_bounded(kv_empty(slot), ((ld / C::kSlots) - 1) & 1u, abort_flag, p);
                             if (!ok) break;
-                        }
-                        tc_fence_after();
-                        issue_pv(t, slot_v, it > 0);
-                        if (it + 1 < g.n[t]) {
-                            if (!k_ready) {
-                                ok = wait_bounded(kv_full(slot_n), (ld_n / C::kSlots) & 1u, abort_flag, p);
-                                if (!ok) break;
-                                k_ready = true;
-                                tc_fence_after();
-                            }
-                            issue_s(t, slot_n);
-                            mma_commit(s_full(t));
-                            if (it + 2 == g.n[t]) mma_commit(q_empty(t));
-                        } else {
-                            mma_commit(o_full(t));
-                            ++on[t];
+                            mbar_arrive_expect_tx(kv_full(slot), (uint32_t)C::kTileBytes);
+#pragma unroll
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes,
+                                            w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v,
+                                            kv_full(slot), c * 64, g.kvh, kpos, g.b);
+                            ++ld;
                         }
                     }
-                    if (!ok) break;
-                    mma_commit(kv_empty(slot_v));
-                    if (next) mma_commit(kv_empty(slot_n));
+                }
+                if (!ok) {
+                    // let the copies already issued land before the CTA's memory is released
+                    const uint32_t first = ld > (uint32_t)C::kSlots ? ld - C::kSlots : 0u;
+                    for (uint32_t l = first; l < ld; ++l)
+                        wait_drain(kv_full(l % C::kSlots), (l / C::kSlots) & 1u, p);
+                    for (int t = 0; t < NT; ++t)
+                        if (qn[t] > 0) wait_drain(q_full(t), (qn[t] - 1) & 1u, p);
                 }
             }
-            // every MMA issued so far must be complete before TMEM is released
-            mma_commit(mma_done);
-            wait_drain(mma_done, 0u, p);
+            __syncwarp();
+        } else if (warp == 1) {
+            // -------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                uint32_t ld = 0;
+                uint32_t qn[NT] = {}, pn[NT] = {}, on[NT] = {};
+                bool ok = true;
+
+                auto issue_s = [&](int t, int slot) {
+                    const uint32_t a0 = sQ + t * C::kTileBytes;
+                    const uint32_t b0 = sKV + slot * C::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < HD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+                        mma_ss(tmem + C::s_col(t), sdesc_sw128(a0 + off, 16, 1024),
+                               sdesc_sw128(b0 + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
+                    }
+                };
+                auto issue_pv = [&](int t, int slot, bool accumulate) {
+                    const uint32_t b0 = sKV + slot * C::kTileBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBlockN / 16; ++kk)
+                        mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
+                               sdesc_sw128(b0 + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
+                               (accumulate || kk > 0) ? 1u : 0u);
+                };
+
+                for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                    const UnitGeom<NT> g = unit_geom<NT>(u, p);
+                    if (g.nblk == 0) continue;
+                    // first key block: S_t for every tile that has keys
+                    int slot_k = ld % C::kSlots;
+                    ok = wait_bounded(kv_full(slot_k), (ld / C::kSlots) & 1u, abort_flag, p);
+                    if (!ok) break;
+                    ++ld;
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        if (g.n[t] == 0 || !ok) continue;
+                        ok = wait_bounded(q_full(t), qn[t] & 1u, abort_flag, p);
+                        if (!ok) break;
+                        ++qn[t];
+                        tc_fence_after();
+                        issue_s(t, slot_k);
+                        mma_commit(s_full(t));
+                        if (g.n[t] == 1) mma_commit(q_empty(t));
+                    }
+                    if (!ok) break;
+                    mma_commit(kv_empty(slot_k));
+
+                    for (int it = 0; it < g.nblk && ok; ++it) {
+                        const int slot_v = ld % C::kSlots;
+                        ok = wait_bounded(kv_full(slot_v), (ld / C::kSlots) & 1u, abort_flag, p);
+                        if (!ok) break;
+                        ++ld;
+                        // K of the next block: waited for only when its first S is issued
+                        const bool next = it + 1 < g.nblk;
+                        const uint32_t ld_n = ld;
+                        const int slot_n = ld_n % C::kSlots;
+                        bool k_ready = false;
+                        if (next) ++ld;
+                        tc_fence_after();
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            if (it >= g.n[t] || !ok) continue;
+                            ok = wait_bounded(p_full(t), pn[t] & 1u, abort_flag, p);
+                            if (!ok) break;
+                            ++pn[t];
+                            if (it == 0 && on[t] > 0) {
+                                // the previous unit's epilogue must have read O_t out
+                                ok = wait_bounded(o_empty(t), (on[t] - 1) & 1u, abort_flag, p);
+                                if (!ok) break;
+                            }
+                            tc_fence_after();
+                            issue_pv(t, slot_v, it > 0);
+                            if (it + 1 < g.n[t]) {
+                                if (!k_ready) {
+                                    ok = wait_bounded(kv_full(slot_n), (ld_n / C::kSlots) & 1u, abort_flag, p);
+                                    if (!ok) break;
+                                    k_ready = true;
+                                    tc_fence_after();
+                                }
+                                issue_s(t, slot_n);
+                                mma_commit(s_full(t));
+                                if (it + 2 == g.n[t]) mma_commit(q_empty(t));
+                            } else {
+                                mma_commit(o_full(t));
+                                ++on[t];
+                            }
+                        }
+                        if (!ok) break;
+                        mma_commit(kv_empty(slot_v));
+                        if (next) mma_commit(kv_empty(slot_n));
+                    }
+                }
+                // every MMA issued so far must be complete before TMEM is released
+                mma_commit(mma_done);
+                wait_drain(mma_done, 0u, p);
+            }
+            __syncwarp();
         }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------------------ softmax warpgroups
-        const int t = (warp - 2) >> 2;
+    } else if (wg <= NT) {
+        // ------------------------------------------------------------ softmax, tile t
+        regs_inc<C::kRegsSoftmax>();
+        const int t = wg - 1;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t s_addr = tl + C::s_col(t);
-        const uint32_t o_addr = tl + C::o_col(t);
-        uint32_t sn = 0, on = 0;
-        bool ok = true;
+        const uint32_t s_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::s_col(t);
+        const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
+        const float c = p.scale_log2;
         const float kNegInf = -INFINITY;
-        constexpr float kLn2 = 0.69314718055994530942f;
+        const float fill = (c >= 0.f) ? -INFINITY : INFINITY;  // masked keys drop out of the extremum
+        uint32_t sn = 0, stn = 0;
+        bool ok = true;
 
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
             const UnitGeom<NT> g = unit_geom<NT>(u, p);
             const int n_t = pick<NT>(g.n, t);
-            const int pos0_t = pick<NT>(g.pos0, t);
-            // row -> (position, head)
-            int pos, head;
-            bool row_ok;
-            if (p.pack) {
-                uint32_t pr, hh;
-                fastdivmod((uint32_t)row, p.div_g, pr, hh);
-                pos = pos0_t + (int)pr;
-                head = g.hg * p.g + (int)hh;
-                row_ok = row < p.rows_valid && pos < p.Sq;
-            } else {
-                pos = pos0_t + row;
-                head = g.hg;
-                row_ok = pos < p.Sq;
-            }
+            if (n_t == 0) continue;
+            const RowMap rm = row_map(p, pick<NT>(g.pos0, t), g.hg, row);
             // exclusive key bound of this row (causal: j <= pos + Sk - Sq)
-            const int kmax = p.causal ? min(p.Sk, pos + 1 + (p.Sk - p.Sq)) : p.Sk;
+            const int kmax = p.causal ? min(p.Sk, rm.pos + 1 + (p.Sk - p.Sq)) : p.Sk;
+            // A warp whose 32 rows are all padding (short query axis, e.g. decode) only
+            // keeps the handshake: its P and O rows feed nothing that is stored.
+            const bool idle = __all_sync(0xffffffffu, !rm.ok);
+            if (idle) {
+                for (int it = 0; it < n_t && ok; ++it) {
+                    ok = __all_sync(0xffffffffu, wait_bounded(s_full(t), sn & 1u, abort_flag, p));
+                    if (!ok) break;
+                    ++sn;
+                    tc_fence_after();
+                    tc_fence_before();
+                    mbar_arrive(p_full(t));
+                }
+                if (!ok) break;
+                ++stn;
+                mbar_arrive(st_full(t));
+                continue;
+            }
 
-            float m = kNegInf;  // reference max, log2 units
+            float m = kNegInf;  // reference max of c*s (log2 units)
             float l = 0.f;
             for (int it = 0; it < n_t; ++it) {
                 ok = __all_sync(0xffffffffu, wait_bounded(s_full(t), sn & 1u, abort_flag, p));
@@ -389,30 +456,41 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 tc_fence_after();
                 float s[128];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int ch = 0; ch < 4; ++ch) {
                     uint32_t r[32];
-                    tmem_ld32(s_addr + c * 32, r);
+                    tmem_ld32(s_addr + ch * 32, r);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 32; ++i) s[ch * 32 + i] = __uint_as_float(r[i]);
                 }
                 tmem_wait_ld();
-                // scores in log2 units, then masking
+                const int lim = kmax - (g.kb_lo + it) * kBlockN;  // keys [0, lim) allowed
+                const bool masked = lim < kBlockN;
+                if (masked) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i) s[i] *= p.scale_log2;
-                const int lim = kmax - (g.kb_lo + it) * kBlockN;
-                if (lim < kBlockN) {
-#pragma unroll
-                    for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : kNegInf;
+                    for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : fill;
                 }
-                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+                // extremum of the raw scores (max for c >= 0, min for c < 0), times c
+                float e0 = s[0], e1 = s[1], e2 = s[2], e3 = s[3];
+                if (c >= 0.f) {
 #pragma unroll
-                for (int i = 4; i < 128; i += 4) {
-                    mx0 = fmaxf(mx0, s[i]);
-                    mx1 = fmaxf(mx1, s[i + 1]);
-                    mx2 = fmaxf(mx2, s[i + 2]);
-                    mx3 = fmaxf(mx3, s[i + 3]);
+                    for (int i = 4; i < 128; i += 4) {
+                        e0 = fmaxf(e0, s[i]);
+                        e1 = fmaxf(e1, s[i + 1]);
+                        e2 = fmaxf(e2, s[i + 2]);
+                        e3 = fmaxf(e3, s[i + 3]);
+                    }
+                    e0 = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));
+                } else {
+#pragma unroll
+                    for (int i = 4; i < 128; i += 4) {
+                        e0 = fminf(e0, s[i]);
+                        e1 = fminf(e1, s[i + 1]);
+                        e2 = fminf(e2, s[i + 2]);
+                        e3 = fminf(e3, s[i + 3]);
+                    }
+                    e0 = fminf(fminf(e0, e1), fminf(e2, e3));
                 }
-                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                const float mx = (lim <= 0) ? kNegInf : (c == 0.f ? 0.f : e0 * c);
                 // Deferred rescaling: move the reference max only when the block's max
                 // exceeds it by more than 8 (a factor 256), which keeps every p <= 256.
                 const bool grow = mx > m + 8.0f;  // false when mx = -inf; true when m = -inf < mx
@@ -422,35 +500,40 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                     l *= alpha;
                     m = mx;
                 }
-                // P = exp2(t - m) as bf16, written over S in TMEM (S is already in registers)
-                const float m_use = (m == kNegInf) ? 0.f : m;
+                // P = 2^(c*s - m) as bf16 over S in TMEM (S is already in registers)
+                const float neg_m = (m == kNegInf) ? 0.f : -m;
                 float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int ch = 0; ch < 4; ++ch) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float p0 = ex2_approx(s[c * 32 + 2 * i] - m_use);
-                        const float p1 = ex2_approx(s[c * 32 + 2 * i + 1] - m_use);
+                        const int j = ch * 32 + 2 * i;
+                        float p0 = ex2_approx(fmaf(s[j], c, neg_m));
+                        float p1 = ex2_approx(fmaf(s[j + 1], c, neg_m));
+                        if (masked) {
+                            p0 = (j < lim) ? p0 : 0.f;
+                            p1 = (j + 1 < lim) ? p1 : 0.f;
+                        }
                         ls0 += p0;
                         ls1 += p1;
                         pk[i] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st16(s_addr + c * 16, pk);
+                    tmem_st16(s_addr + ch * 16, pk);
                 }
                 l += ls0 + ls1;
                 // O rescale (after P, so the S registers are free): PV of the previous
                 // block is complete, because this block's S was issued after it.
                 if (it > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
+                    for (int ch = 0; ch < HD / 32; ++ch) {
                         uint32_t r[32];
-                        tmem_ld32(o_addr + c * 32, r);
+                        tmem_ld32(o_addr + ch * 32, r);
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                        tmem_st32(o_addr + c * 32, r);
+                        tmem_st32(o_addr + ch * 32, r);
                     }
                 }
                 tmem_wait_st();
@@ -458,51 +541,85 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 mbar_arrive(p_full(t));
             }
             if (!ok) break;
-
-            // ---------------------------------------------------------- epilogue
-            const bool has = n_t > 0;
-            if (has) {
-                ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), on & 1u, abort_flag, p));
+            // row statistics for the epilogue warpgroup (double-buffered by unit)
+            float* st = stats + ((stn & 1u) * NT + t) * 256;
+            st[row] = m;
+            st[128 + row] = l;
+            ++stn;
+            mbar_arrive(st_full(t));
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        if constexpr (C::kRegsEpilogue < C::kLaunchRegs) regs_dec<C::kRegsEpilogue>();
+        if constexpr (C::kRegsEpilogue > C::kLaunchRegs) regs_inc<C::kRegsEpilogue>();
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const float kNegInf = -INFINITY;
+        constexpr float kLn2 = 0.69314718055994530942f;
+        uint32_t on[NT] = {}, stn[NT] = {};
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+            const UnitGeom<NT> g = unit_geom<NT>(u, p);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
                 if (!ok) break;
-                ++on;
-                tc_fence_after();
-            }
-            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : kNegInf;
-            float* orow;
-            float* lrow;
-            if (p.num_splits == 1) {
-                orow = p.out + (((size_t)g.b * p.Sq + pos) * p.Hq + head) * HD;
-                lrow = p.lse + ((size_t)g.b * p.Hq + head) * p.Sq + pos;
-            } else {
-                const size_t r = (((size_t)g.split * p.B + g.b) * p.Hq + head) * p.Sq + pos;
-                orow = p.o_part + r * HD;
-                lrow = p.lse_part + r;
-            }
-#pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-                uint32_t r[32];
+                const RowMap rm = row_map(p, g.pos0[t], g.hg, row);
+                const bool has = g.n[t] > 0;
+                const bool idle = __all_sync(0xffffffffu, !rm.ok);
+                float m = kNegInf, l = 0.f;
                 if (has) {
-                    tmem_ld32(o_addr + c * 32, r);
-                    tmem_wait_ld();
+                    ok = __all_sync(0xffffffffu, wait_bounded(st_full(t), stn[t] & 1u, abort_flag, p));
+                    if (!ok) break;
+                    const float* st = stats + ((stn[t] & 1u) * NT + t) * 256;
+                    m = st[row];
+                    l = st[128 + row];
+                    ++stn[t];
+                    ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), on[t] & 1u, abort_flag, p));
+                    if (!ok) break;
+                    ++on[t];
+                    tc_fence_after();
                 }
-                if (row_ok) {
-                    float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : kNegInf;
+                float* orow;
+                float* lrow;
+                if (p.num_splits == 1) {
+                    orow = p.out + (((size_t)g.b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
+                    lrow = p.lse + ((size_t)g.b * p.Hq + rm.head) * p.Sq + rm.pos;
+                } else {
+                    const size_t r = (((size_t)g.split * p.B + g.b) * p.Hq + rm.head) * p.Sq + rm.pos;
+                    orow = p.o_part + r * HD;
+                    lrow = p.lse_part + r;
+                }
+                const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        float4 v;
-                        v.x = has ? __uint_as_float(r[4 * i + 0]) * inv_l : 0.f;
-                        v.y = has ? __uint_as_float(r[4 * i + 1]) * inv_l : 0.f;
-                        v.z = has ? __uint_as_float(r[4 * i + 2]) * inv_l : 0.f;
-                        v.w = has ? __uint_as_float(r[4 * i + 3]) * inv_l : 0.f;
-                        dst[i] = v;
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    uint32_t r[32];
+                    if (has) {
+                        if (!idle) {
+                            tmem_ld32(o_addr + ch * 32, r);
+                            tmem_wait_ld();
+                        }
+                        if (ch == HD / 32 - 1) {
+                            // O_t is in registers: the next unit's PV may overwrite it
+                            tc_fence_before();
+                            mbar_arrive(o_empty(t));
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = 0u;
+                    }
+                    if (rm.ok) {
+                        float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l,
+                                                 __uint_as_float(r[4 * i + 1]) * inv_l,
+                                                 __uint_as_float(r[4 * i + 2]) * inv_l,
+                                                 __uint_as_float(r[4 * i + 3]) * inv_l);
                     }
                 }
-            }
-            if (row_ok) *lrow = lse_v;
-            if (has) {
-                tc_fence_before();
-                mbar_arrive(o_empty(t));
+                if (rm.ok) *lrow = lse_v;
             }
         }
     }
@@ -585,6 +702,16 @@ cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
+    // setmaxnreg redistributes the registers the CTA was launched with: refuse to launch
+    // a build whose register count differs from the split's assumption
+    static int regs_checked = 0;  // 0 unknown, 1 ok, -1 mismatch
+    if (regs_checked == 0) {
+        cudaFuncAttributes attr{};
+        cudaError_t e = cudaFuncGetAttributes(&attr, gqa_fwd_kernel<HD, NT>);
+        if (e != cudaSuccess) return e;
+        regs_checked = (attr.numRegs == C::kLaunchRegs) ? 1 : -1;
+    }
+    if (regs_checked != 1) return cudaErrorInvalidConfiguration;
     gqa_fwd_kernel<HD, NT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
     return cudaGetLastError();
 }
