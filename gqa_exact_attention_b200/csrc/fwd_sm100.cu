@@ -40,26 +40,31 @@ struct FwdCfg {
     static constexpr int kChunks = HD / 64;              // 128-byte column chunks of a row
     static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kSlots = (NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 5 : 10);
-    // warpgroups: 0 = TMA producer + MMA issuer, 1..NT = softmax (one per tile),
-    // NT+1 = epilogue
-    static constexpr int kWarpgroups = 2 + NT;
+    static constexpr int kSlots = (NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 2 : 5);
+    // NT == 2: warpgroups 0 = TMA producer + MMA issuer, 1..2 = softmax (one per tile),
+    //          3 = epilogue; one CTA per SM.
+    // NT == 1: warpgroup 0 as above, 1 = softmax that also writes its tile's output; two
+    //          CTAs per SM, so one CTA's unit changes overlap the other's K/V stream.
+    static constexpr bool kEpilogueWG = (NT == 2);
+    static constexpr int kWarpgroups = 1 + NT + (kEpilogueWG ? 1 : 0);
     static constexpr int kThreads = kWarpgroups * 128;
-    static constexpr int kCtasPerSm = 1;
-    // registers: at launch (65536 / threads, rounded down to 8), then redistributed with
-    // setmaxnreg; the per-thread sum over the warpgroups equals warpgroups x launch regs,
-    // so every increase is covered by the decreases (each sub-partition holds one warp of
-    // each warpgroup)
-    static constexpr int kLaunchRegs = ((65536 / kThreads) / 8) * 8;
+    static constexpr int kCtasPerSm = kEpilogueWG ? 1 : 2;
+    // registers: at launch (65536 / (threads x CTAs), rounded down to 8), then
+    // redistributed with setmaxnreg; the per-thread sum over the warpgroups equals
+    // warpgroups x launch regs, so every increase is covered by the decreases (each SM
+    // sub-partition holds one warp of each warpgroup)
+    static constexpr int kLaunchRegs = ((65536 / (kThreads * kCtasPerSm)) / 8) * 8;
     static constexpr int kRegsLoad = NT == 2 ? 96 : 56;
-    static constexpr int kRegsSoftmax = NT == 2 ? 168 : 232;
-    static constexpr int kRegsEpilogue = kWarpgroups * kLaunchRegs - kRegsLoad - NT * kRegsSoftmax;
+    static constexpr int kRegsSoftmax = NT == 2 ? 168 : 200;
+    static constexpr int kRegsEpilogue =
+        kEpilogueWG ? kWarpgroups * kLaunchRegs - kRegsLoad - NT * kRegsSoftmax : 0;
     static_assert(kRegsLoad + NT * kRegsSoftmax + kRegsEpilogue == kWarpgroups * kLaunchRegs,
                   "register split must add up to the launch allocation");
-    static_assert(kRegsEpilogue >= 64 && kRegsEpilogue % 8 == 0, "epilogue registers");
+    static_assert(!kEpilogueWG || (kRegsEpilogue >= 64 && kRegsEpilogue % 8 == 0),
+                  "epilogue registers");
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
     static constexpr int kNumBars = 2 * kSlots + 7 * NT + 1;
-    static constexpr int kStatsBytes = 2 * NT * 2 * 128 * 4;  // (m, l) per row, 2 buffers
+    static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + NT * kTileBytes +
                                       kSlots * kTileBytes + 8 * kNumBars + kStatsBytes + 16;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -164,6 +169,55 @@ __device__ __forceinline__ RowMap row_map(const FwdParams& p, int pos0, int hg, 
     return m;
 }
 
+// Writes one tile row's output: O / l from TMEM (or zeros for a tile with no key in this
+// split) and LSE = (m + log2 l) ln 2, to out/lse or to the split partials.  Arrives on
+// o_empty once O is in registers, so the next unit's PV may overwrite it.
+template <int HD>
+__device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, const RowMap& rm,
+                                          int b, int split, bool has, bool idle, float m, float l,
+                                          uint32_t o_empty_bar) {
+    constexpr float kLn2 = 0.69314718055994530942f;
+    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
+    float* orow;
+    float* lrow;
+    if (p.num_splits == 1) {
+        orow = p.out + (((size_t)b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
+        lrow = p.lse + ((size_t)b * p.Hq + rm.head) * p.Sq + rm.pos;
+    } else {
+        const size_t r = (((size_t)split * p.B + b) * p.Hq + rm.head) * p.Sq + rm.pos;
+        orow = p.o_part + r * HD;
+        lrow = p.lse_part + r;
+    }
+#pragma unroll
+    for (int ch = 0; ch < HD / 32; ++ch) {
+        uint32_t r[32];
+        if (has) {
+            if (!idle) {
+                ptx::tmem_ld32(o_addr + ch * 32, r);
+                ptx::tmem_wait_ld();
+            }
+            if (ch == HD / 32 - 1) {
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(o_empty_bar);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = 0u;
+        }
+        if (rm.ok) {
+            float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l,
+                                     __uint_as_float(r[4 * i + 1]) * inv_l,
+                                     __uint_as_float(r[4 * i + 2]) * inv_l,
+                                     __uint_as_float(r[4 * i + 3]) * inv_l);
+        }
+    }
+    if (rm.ok) *lrow = lse_v;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting or when
 // this wait ran past the time limit (then it records the timeout and starts the abort).
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
@@ -194,7 +248,7 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const 
 }
 
 template <int HD, int NT>
-__global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCtasPerSm)
     gqa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<HD, NT>;
     extern __shared__ uint8_t smem_raw[];
@@ -206,7 +260,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
     const uint32_t sKV = base + NT * C::kTileBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NT * C::kTileBytes + C::kSlots * C::kTileBytes);
     float* stats = reinterpret_cast<float*>(bars + C::kNumBars);  // [2][NT][2][128]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stats + 2 * NT * 2 * 128);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(stats) + C::kStatsBytes);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const uint32_t bar0 = smem_u32(bars);
@@ -419,14 +473,18 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
         const float c = p.scale_log2;
         const float kNegInf = -INFINITY;
         const float fill = (c >= 0.f) ? -INFINITY : INFINITY;  // masked keys drop out of the extremum
-        uint32_t sn = 0, stn = 0;
+        uint32_t sn = 0, stn = 0, sn_o = 0;
         bool ok = true;
 
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
             const UnitGeom<NT> g = unit_geom<NT>(u, p);
             const int n_t = pick<NT>(g.n, t);
-            if (n_t == 0) continue;
             const RowMap rm = row_map(p, pick<NT>(g.pos0, t), g.hg, row);
+            if (n_t == 0) {
+                if constexpr (!C::kEpilogueWG)
+                    write_row<HD>(p, o_addr, rm, g.b, g.split, false, true, -INFINITY, 0.f, 0u);
+                continue;
+            }
             // exclusive key bound of this row (causal: j <= pos + Sk - Sq)
             const int kmax = p.causal ? min(p.Sk, rm.pos + 1 + (p.Sk - p.Sq)) : p.Sk;
             // A warp whose 32 rows are all padding (short query axis, e.g. decode) only
@@ -442,8 +500,16 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
                     mbar_arrive(p_full(t));
                 }
                 if (!ok) break;
-                ++stn;
-                mbar_arrive(st_full(t));
+                if constexpr (C::kEpilogueWG) {
+                    ++stn;
+                    mbar_arrive(st_full(t));
+                } else {
+                    ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), sn_o & 1u, abort_flag, p));
+                    if (!ok) break;
+                    ++sn_o;
+                    tc_fence_after();
+                    write_row<HD>(p, o_addr, rm, g.b, g.split, true, true, kNegInf, 0.f, o_empty(t));
+                }
                 continue;
             }
 
@@ -541,21 +607,27 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
                 mbar_arrive(p_full(t));
             }
             if (!ok) break;
-            // row statistics for the epilogue warpgroup (double-buffered by unit)
-            float* st = stats + ((stn & 1u) * NT + t) * 256;
-            st[row] = m;
-            st[128 + row] = l;
-            ++stn;
-            mbar_arrive(st_full(t));
+            if constexpr (C::kEpilogueWG) {
+                // row statistics for the epilogue warpgroup (double-buffered by unit)
+                float* st = stats + ((stn & 1u) * NT + t) * 256;
+                st[row] = m;
+                st[128 + row] = l;
+                ++stn;
+                mbar_arrive(st_full(t));
+            } else {
+                ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), sn_o & 1u, abort_flag, p));
+                if (!ok) break;
+                ++sn_o;
+                tc_fence_after();
+                write_row<HD>(p, o_addr, rm, g.b, g.split, true, false, m, l, o_empty(t));
+            }
         }
-    } else {
+    } else if constexpr (C::kEpilogueWG) {
         // ------------------------------------------------------------ epilogue
         if constexpr (C::kRegsEpilogue < C::kLaunchRegs) regs_dec<C::kRegsEpilogue>();
         if constexpr (C::kRegsEpilogue > C::kLaunchRegs) regs_inc<C::kRegsEpilogue>();
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const float kNegInf = -INFINITY;
-        constexpr float kLn2 = 0.69314718055994530942f;
         uint32_t on[NT] = {}, stn[NT] = {};
         bool ok = true;
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -566,7 +638,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
                 const RowMap rm = row_map(p, g.pos0[t], g.hg, row);
                 const bool has = g.n[t] > 0;
                 const bool idle = __all_sync(0xffffffffu, !rm.ok);
-                float m = kNegInf, l = 0.f;
+                float m = -INFINITY, l = 0.f;
                 if (has) {
                     ok = __all_sync(0xffffffffu, wait_bounded(st_full(t), stn[t] & 1u, abort_flag, p));
                     if (!ok) break;
@@ -579,47 +651,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, 1)
                     ++on[t];
                     tc_fence_after();
                 }
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : kNegInf;
-                float* orow;
-                float* lrow;
-                if (p.num_splits == 1) {
-                    orow = p.out + (((size_t)g.b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
-                    lrow = p.lse + ((size_t)g.b * p.Hq + rm.head) * p.Sq + rm.pos;
-                } else {
-                    const size_t r = (((size_t)g.split * p.B + g.b) * p.Hq + rm.head) * p.Sq + rm.pos;
-                    orow = p.o_part + r * HD;
-                    lrow = p.lse_part + r;
-                }
                 const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
-#pragma unroll
-                for (int ch = 0; ch < HD / 32; ++ch) {
-                    uint32_t r[32];
-                    if (has) {
-                        if (!idle) {
-                            tmem_ld32(o_addr + ch * 32, r);
-                            tmem_wait_ld();
-                        }
-                        if (ch == HD / 32 - 1) {
-                            // O_t is in registers: the next unit's PV may overwrite it
-                            tc_fence_before();
-                            mbar_arrive(o_empty(t));
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) r[i] = 0u;
-                    }
-                    if (rm.ok) {
-                        float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(__uint_as_float(r[4 * i + 0]) * inv_l,
-                                                 __uint_as_float(r[4 * i + 1]) * inv_l,
-                                                 __uint_as_float(r[4 * i + 2]) * inv_l,
-                                                 __uint_as_float(r[4 * i + 3]) * inv_l);
-                    }
-                }
-                if (rm.ok) *lrow = lse_v;
+                write_row<HD>(p, o_addr, rm, g.b, g.split, has, idle, m, l, o_empty(t));
             }
         }
     }
