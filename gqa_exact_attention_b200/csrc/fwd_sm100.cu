@@ -315,17 +315,20 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
         regs_dec<C::kRegsLoad>();
         if (warp == 0) {
             // -------------------------------------------------------- TMA producer
-            if (lane == 0) {
-                uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
-                uint32_t qn[NT] = {};  // Q loads issued per tile
-                bool ok = true;
-                for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                    const UnitGeom<NT> g = unit_geom<NT>(u, p);
+            // The whole warp runs the loop (so its values stay warp-uniform); one elected
+            // lane issues the copies.
+            uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
+            uint32_t qn[NT] = {};  // Q loads issued per tile
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const UnitGeom<NT> g = unit_geom<NT>(u, p);
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        if (g.n[t] == 0 || !ok) continue;
-                        if (qn[t] > 0) ok = wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p);
-                        if (!ok) break;
+                for (int t = 0; t < NT; ++t) {
+                    if (g.n[t] == 0 || !ok) continue;
+                    if (qn[t] > 0)
+                        ok = __all_sync(0xffffffffu, wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p));
+                    if (!ok) break;
+                    if (elect_one()) {
                         const int rows = p.pack ? p.rows_valid : kBlockM;
                         mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
                         const int hcoord = p.pack ? g.hg * p.g : g.hg;
@@ -333,133 +336,185 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                         for (int c = 0; c < C::kChunks; ++c)
                             tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
                                         q_full(t), c * 64, hcoord, g.pos0[t], g.b);
-                        ++qn[t];
                     }
-                    for (int it = 0; it < g.nblk && ok; ++it) {
-                        const int kpos = (g.kb_lo + it) * kBlockN;
+                    __syncwarp();
+                    ++qn[t];
+                }
+                for (int it = 0; it < g.nblk && ok; ++it) {
+                    const int kpos = (g.kb_lo + it) * kBlockN;
 #pragma unroll
-                        for (int w = 0; w < 2; ++w) {
-                            const int slot = ld % C::kSlots;
-                            if (ld >= (uint32_t)C::kSlots)
-                                ok = wait_bounded(kv_empty(slot), ((ld / C::kSlots) - 1) & 1u, abort_flag, p);
-                            if (!ok) break;
+                    for (int w = 0; w < 2; ++w) {
+                        const int slot = ld % C::kSlots;
+                        if (ld >= (uint32_t)C::kSlots)
+                            ok = __all_sync(0xffffffffu, wait_bounded(kv_empty(slot), ((ld / C::kSlots) - 1) & 1u, abort_flag, p));
+                        if (!ok) break;
+                        if (elect_one()) {
                             mbar_arrive_expect_tx(kv_full(slot), (uint32_t)C::kTileBytes);
 #pragma unroll
                             for (int c = 0; c < C::kChunks; ++c)
                                 tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes,
                                             w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v,
                                             kv_full(slot), c * 64, g.kvh, kpos, g.b);
-                            ++ld;
                         }
+                        __syncwarp();
+                        ++ld;
                     }
                 }
-                if (!ok) {
-                    // let the copies already issued land before the CTA's memory is released
-                    const uint32_t first = ld > (uint32_t)C::kSlots ? ld - C::kSlots : 0u;
-                    for (uint32_t l = first; l < ld; ++l)
-                        wait_drain(kv_full(l % C::kSlots), (l / C::kSlots) & 1u, p);
-                    for (int t = 0; t < NT; ++t)
-                        if (qn[t] > 0) wait_drain(q_full(t), (qn[t] - 1) & 1u, p);
-                }
+            }
+            if (!ok) {
+                // let the copies already issued land before the CTA's memory is released
+                const uint32_t first = ld > (uint32_t)C::kSlots ? ld - C::kSlots : 0u;
+                for (uint32_t l = first; l < ld; ++l)
+                    wait_drain(kv_full(l % C::kSlots), (l / C::kSlots) & 1u, p);
+                for (int t = 0; t < NT; ++t)
+                    if (qn[t] > 0) wait_drain(q_full(t), (qn[t] - 1) & 1u, p);
             }
             __syncwarp();
         } else if (warp == 1) {
             // -------------------------------------------------------- MMA issuer
-            if (lane == 0) {
-                uint32_t ld = 0;
-                uint32_t qn[NT] = {}, pn[NT] = {}, on[NT] = {};
-                bool ok = true;
-
-                auto issue_s = [&](int t, int slot) {
-                    const uint32_t a0 = sQ + t * C::kTileBytes;
-                    const uint32_t b0 = sKV + slot * C::kTileBytes;
+            // The whole warp runs the loop: barrier waits and descriptors are warp-uniform,
+            // and one elected lane issues each group of MMAs and its commit.
+            uint32_t ld = 0;
+            uint32_t qn[NT] = {}, pn[NT] = {}, on[NT] = {};
+            bool ok = true;
+            // descriptors built once; each MMA advances them by a constant offset
+            const uint64_t q_desc0 = sdesc_sw128(sQ, 16, 1024);
+            const uint64_t k_desc0 = sdesc_sw128(sKV, 16, 1024);
+            const uint64_t v_desc0 = sdesc_sw128(sKV, C::kChunkBytes, 1024);
+            // Issue a group of MMAs; before its last MMA, probe (without blocking) the
+            // barrier the next group will wait on, so the probe's latency overlaps that
+            // MMA instead of leaving the tensor pipe idle.  Returns the probe's result.
+            auto issue_s = [&](int t, int slot, uint32_t probe_bar, uint32_t probe_par) {
+                const uint64_t a0 = sdesc_add(q_desc0, t * C::kTileBytes);
+                const uint64_t b0 = sdesc_add(k_desc0, slot * C::kTileBytes);
+                const uint32_t d = tmem + C::s_col(t);
+                bool ready = false;
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < HD / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                        mma_ss(tmem + C::s_col(t), sdesc_sw128(a0 + off, 16, 1024),
-                               sdesc_sw128(b0 + off, 16, 1024), C::kIdescQK, kk > 0 ? 1u : 0u);
-                    }
-                };
-                auto issue_pv = [&](int t, int slot, bool accumulate) {
-                    const uint32_t b0 = sKV + slot * C::kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk)
-                        mma_ts(tmem + C::o_col(t), tmem + C::s_col(t) + kk * 8,
-                               sdesc_sw128(b0 + kk * 2048, C::kChunkBytes, 1024), C::kIdescPV,
-                               (accumulate || kk > 0) ? 1u : 0u);
-                };
-
-                for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-                    const UnitGeom<NT> g = unit_geom<NT>(u, p);
-                    if (g.nblk == 0) continue;
-                    // first key block: S_t for every tile that has keys
-                    int slot_k = ld % C::kSlots;
-                    ok = wait_bounded(kv_full(slot_k), (ld / C::kSlots) & 1u, abort_flag, p);
-                    if (!ok) break;
-                    ++ld;
-#pragma unroll
-                    for (int t = 0; t < NT; ++t) {
-                        if (g.n[t] == 0 || !ok) continue;
-                        ok = wait_bounded(q_full(t), qn[t] & 1u, abort_flag, p);
-                        if (!ok) break;
-                        ++qn[t];
-                        tc_fence_after();
-                        issue_s(t, slot_k);
-                        mma_commit(s_full(t));
-                        if (g.n[t] == 1) mma_commit(q_empty(t));
-                    }
-                    if (!ok) break;
-                    mma_commit(kv_empty(slot_k));
-
-                    for (int it = 0; it < g.nblk && ok; ++it) {
-                        const int slot_v = ld % C::kSlots;
-                        ok = wait_bounded(kv_full(slot_v), (ld / C::kSlots) & 1u, abort_flag, p);
-                        if (!ok) break;
-                        ++ld;
-                        // K of the next block: waited for only when its first S is issued
-                        const bool next = it + 1 < g.nblk;
-                        const uint32_t ld_n = ld;
-                        const int slot_n = ld_n % C::kSlots;
-                        bool k_ready = false;
-                        if (next) ++ld;
-                        tc_fence_after();
-#pragma unroll
-                        for (int t = 0; t < NT; ++t) {
-                            if (it >= g.n[t] || !ok) continue;
-                            ok = wait_bounded(p_full(t), pn[t] & 1u, abort_flag, p);
-                            if (!ok) break;
-                            ++pn[t];
-                            if (it == 0 && on[t] > 0) {
-                                // the previous unit's epilogue must have read O_t out
-                                ok = wait_bounded(o_empty(t), (on[t] - 1) & 1u, abort_flag, p);
-                                if (!ok) break;
-                            }
-                            tc_fence_after();
-                            issue_pv(t, slot_v, it > 0);
-                            if (it + 1 < g.n[t]) {
-                                if (!k_ready) {
-                                    ok = wait_bounded(kv_full(slot_n), (ld_n / C::kSlots) & 1u, abort_flag, p);
-                                    if (!ok) break;
-                                    k_ready = true;
-                                    tc_fence_after();
-                                }
-                                issue_s(t, slot_n);
-                                mma_commit(s_full(t));
-                                if (it + 2 == g.n[t]) mma_commit(q_empty(t));
-                            } else {
-                                mma_commit(o_full(t));
-                                ++on[t];
-                            }
-                        }
-                        if (!ok) break;
-                        mma_commit(kv_empty(slot_v));
-                        if (next) mma_commit(kv_empty(slot_n));
+                        if (kk == HD / 16 - 1 && probe_bar != 0u) ready = mbar_test_wait(probe_bar, probe_par);
+                        mma_ss(d, sdesc_add(a0, off), sdesc_add(b0, off), C::kIdescQK,
+                               kk > 0 ? 1u : 0u);
                     }
                 }
-                // every MMA issued so far must be complete before TMEM is released
-                mma_commit(mma_done);
-                wait_drain(mma_done, 0u, p);
+                return __ballot_sync(0xffffffffu, ready) != 0u;  // only the issuing lane probed
+            };
+            // O_t += P_t V over the block's 128 keys
+            auto issue_pv = [&](int t, int slot, bool accumulate, uint32_t probe_bar,
+                                uint32_t probe_par) {
+                const uint64_t b0 = sdesc_add(v_desc0, slot * C::kTileBytes);
+                const uint32_t d = tmem + C::o_col(t);
+                const uint32_t a = tmem + C::s_col(t);
+                bool ready = false;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                        if (kk == kBlockN / 16 - 1 && probe_bar != 0u) ready = mbar_test_wait(probe_bar, probe_par);
+                        mma_ts(d, a + kk * 8, sdesc_add(b0, kk * 2048), C::kIdescPV,
+                               (accumulate || kk > 0) ? 1u : 0u);
+                    }
+                }
+                return __ballot_sync(0xffffffffu, ready) != 0u;  // only the issuing lane probed
+            };
+            auto commit = [&](uint32_t bar) {
+                if (elect_one()) mma_commit(bar);
+                __syncwarp();
+            };
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p));
+            };
+
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const UnitGeom<NT> g = unit_geom<NT>(u, p);
+                if (g.nblk == 0) continue;
+                // first key block: S_t for every tile that has keys
+                int slot_k = ld % C::kSlots;
+                ok = wait(kv_full(slot_k), (ld / C::kSlots) & 1u);
+                if (!ok) break;
+                ++ld;
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (g.n[t] == 0 || !ok) continue;
+                    ok = wait(q_full(t), qn[t] & 1u);
+                    if (!ok) break;
+                    ++qn[t];
+                    tc_fence_after();
+                    issue_s(t, slot_k, 0u, 0u);
+                    commit(s_full(t));
+                    if (g.n[t] == 1) commit(q_empty(t));
+                }
+                if (!ok) break;
+                commit(kv_empty(slot_k));
+
+                bool v_ready = false;  // the next V block's barrier was already seen complete
+                for (int it = 0; it < g.nblk && ok; ++it) {
+                    const int slot_v = ld % C::kSlots;
+                    if (!v_ready) ok = wait(kv_full(slot_v), (ld / C::kSlots) & 1u);
+                    if (!ok) break;
+                    ++ld;
+                    // K of the next block: waited for only when its first S is issued
+                    const bool next = it + 1 < g.nblk;
+                    const uint32_t ld_n = ld;
+                    const int slot_n = ld_n % C::kSlots;
+                    const uint32_t kbar = kv_full(slot_n), kpar = (ld_n / C::kSlots) & 1u;
+                    bool k_ready = false;
+                    if (next) ++ld;
+                    // the V block after next: probed at the end of this iteration
+                    const uint32_t vbar = next ? kv_full(ld % C::kSlots) : 0u;
+                    const uint32_t vpar = (ld / C::kSlots) & 1u;
+                    v_ready = false;
+                    tc_fence_after();
+                    bool p_ready = false;  // this tile's P was already seen complete
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        if (it >= g.n[t] || !ok) continue;
+                        if (!p_ready) ok = wait(p_full(t), pn[t] & 1u);
+                        if (!ok) break;
+                        ++pn[t];
+                        if (it == 0 && on[t] > 0) {
+                            // the previous unit's epilogue must have read O_t out
+                            ok = wait(o_empty(t), (on[t] - 1) & 1u);
+                            if (!ok) break;
+                        }
+                        tc_fence_after();
+                        const bool more = it + 1 < g.n[t];
+                        // probe what comes next: this tile's next K, else the next tile's P
+                        const bool has_next_tile = (t + 1 < NT) && (it < g.n[t + 1 < NT ? t + 1 : t]);
+                        const uint32_t pbar_next = has_next_tile ? p_full(t + 1 < NT ? t + 1 : t) : 0u;
+                        const uint32_t ppar_next = has_next_tile ? (pn[t + 1 < NT ? t + 1 : t] & 1u) : 0u;
+                        bool probed = issue_pv(t, slot_v, it > 0,
+                                               more && !k_ready ? kbar : pbar_next,
+                                               more && !k_ready ? kpar : ppar_next);
+                        if (more) {
+                            if (!k_ready) {
+                                if (!probed) ok = wait(kbar, kpar);
+                                if (!ok) break;
+                                k_ready = true;
+                                tc_fence_after();
+                            }
+                            p_ready = issue_s(t, slot_n, has_next_tile ? pbar_next : vbar,
+                                              has_next_tile ? ppar_next : vpar);
+                            if (!has_next_tile) {
+                                v_ready = p_ready;
+                                p_ready = false;
+                            }
+                            commit(s_full(t));
+                            if (it + 2 == g.n[t]) commit(q_empty(t));
+                        } else {
+                            p_ready = has_next_tile && probed;
+                            commit(o_full(t));
+                            ++on[t];
+                        }
+                    }
+                    if (!ok) break;
+                    commit(kv_empty(slot_v));
+                    if (next) commit(kv_empty(slot_n));
+                }
             }
+            // every MMA issued so far must be complete before TMEM is released
+            commit(mma_done);
+            wait_drain(mma_done, 0u, p);
             __syncwarp();
         }
     } else if (wg <= NT) {
@@ -535,28 +590,56 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
 #pragma unroll
                     for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : fill;
                 }
-                // extremum of the raw scores (max for c >= 0, min for c < 0), times c
-                float e0 = s[0], e1 = s[1], e2 = s[2], e3 = s[3];
+                // P = 2^(c*s - m) against the current reference max m, computed before
+                // the block's own max is known (that max only decides whether m has to
+                // move, which is rare after a row's first block).  First half: 64 keys.
+                float neg_m = (m == kNegInf) ? 0.f : -m;
+                float ls0 = 0.f, ls1 = 0.f;
+                // exponentials of keys [32*ch0, 32*ch1), packed to bf16 and stored over S
+                auto exp_range = [&](int ch0, int ch1) {
+#pragma unroll
+                    for (int ch = ch0; ch < ch1; ++ch) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int j = ch * 32 + 2 * i;
+                            float x0, x1;
+                            fma2(s[j], s[j + 1], c, c, neg_m, neg_m, x0, x1);
+                            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            if (masked) {
+                                p0 = (j < lim) ? p0 : 0.f;
+                                p1 = (j + 1 < lim) ? p1 : 0.f;
+                            }
+                            add2(ls0, ls1, p0, p1, ls0, ls1);
+                            pk[i] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(s_addr + ch * 16, pk);
+                    }
+                };
+                if (it > 0) exp_range(0, 2);
+                // extremum of the raw scores (max for c >= 0, min for c < 0), times c:
+                // eight chains of three-input max/min
+                float e[8];
                 if (c >= 0.f) {
 #pragma unroll
-                    for (int i = 4; i < 128; i += 4) {
-                        e0 = fmaxf(e0, s[i]);
-                        e1 = fmaxf(e1, s[i + 1]);
-                        e2 = fmaxf(e2, s[i + 2]);
-                        e3 = fmaxf(e3, s[i + 3]);
+                    for (int k = 0; k < 8; ++k) {
+                        e[k] = max3(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+                        for (int i = 3; i < 15; i += 2) e[k] = max3(e[k], s[k + 8 * i], s[k + 8 * i + 8]);
+                        e[k] = fmaxf(e[k], s[k + 120]);
                     }
-                    e0 = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3));
+                    e[0] = fmaxf(max3(e[0], e[1], e[2]), max3(e[3], e[4], max3(e[5], e[6], e[7])));
                 } else {
 #pragma unroll
-                    for (int i = 4; i < 128; i += 4) {
-                        e0 = fminf(e0, s[i]);
-                        e1 = fminf(e1, s[i + 1]);
-                        e2 = fminf(e2, s[i + 2]);
-                        e3 = fminf(e3, s[i + 3]);
+                    for (int k = 0; k < 8; ++k) {
+                        e[k] = min3(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+                        for (int i = 3; i < 15; i += 2) e[k] = min3(e[k], s[k + 8 * i], s[k + 8 * i + 8]);
+                        e[k] = fminf(e[k], s[k + 120]);
                     }
-                    e0 = fminf(fminf(e0, e1), fminf(e2, e3));
+                    e[0] = fminf(min3(e[0], e[1], e[2]), min3(e[3], e[4], min3(e[5], e[6], e[7])));
                 }
-                const float mx = (lim <= 0) ? kNegInf : (c == 0.f ? 0.f : e0 * c);
+                const float mx = (lim <= 0) ? kNegInf : (c == 0.f ? 0.f : e[0] * c);
                 // Deferred rescaling: move the reference max only when the block's max
                 // exceeds it by more than 8 (a factor 256), which keeps every p <= 256.
                 const bool grow = mx > m + 8.0f;  // false when mx = -inf; true when m = -inf < mx
@@ -565,31 +648,16 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                     alpha = (m == kNegInf) ? 0.f : ex2_approx(m - mx);
                     l *= alpha;
                     m = mx;
+                    neg_m = -m;
                 }
-                // P = 2^(c*s - m) as bf16 over S in TMEM (S is already in registers)
-                const float neg_m = (m == kNegInf) ? 0.f : -m;
-                float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int j = ch * 32 + 2 * i;
-                        float p0 = ex2_approx(fmaf(s[j], c, neg_m));
-                        float p1 = ex2_approx(fmaf(s[j + 1], c, neg_m));
-                        if (masked) {
-                            p0 = (j < lim) ? p0 : 0.f;
-                            p1 = (j + 1 < lim) ? p1 : 0.f;
-                        }
-                        ls0 += p0;
-                        ls1 += p1;
-                        pk[i] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st16(s_addr + ch * 16, pk);
+                if (it == 0 || __any_sync(0xffffffffu, grow)) {
+                    // (re)compute the first half against the moved reference max
+                    ls0 = 0.f;
+                    ls1 = 0.f;
+                    exp_range(0, 2);
                 }
-                l += ls0 + ls1;
-                // O rescale (after P, so the S registers are free): PV of the previous
-                // block is complete, because this block's S was issued after it.
+                // O rescale before the first P.V of this block: PV of the previous block
+                // is complete, because this block's S was issued after it.
                 if (it > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
                     for (int ch = 0; ch < HD / 32; ++ch) {
@@ -602,6 +670,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                         tmem_st32(o_addr + ch * 32, r);
                     }
                 }
+                // second half: keys 64..127
+                exp_range(2, 4);
+                l += ls0 + ls1;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(p_full(t));
