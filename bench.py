@@ -181,12 +181,20 @@ def barrier(pg):
 
 
 def max_over_ranks(pg, x):
+    """Max of a per-rank float over all ranks (the slowest rank sets the job's time)."""
     if pg is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if pg.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(per_rank_work, world, total_ms, steps):
+    """Whole-job rate: every rank processes per_rank_work per step (weak scaling), and
+    the job's time per step is the slowest rank's."""
+    return world * per_rank_work / (total_ms / steps / 1e3)
 
 
 # ----------------------------------------------------------------- CPU oracle timing
@@ -326,7 +334,7 @@ def run_gpu(args, cfg):
         achieved = by / (launch_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-        value = world * by / (ms_per_step / 1e3) / 1e9
+        value = job_throughput(by, world, total_ms, args.steps) / 1e9
         unit = "GB/s"
         e2e_value = world * by / (e2e_ms / 1e3) / 1e9
     else:
@@ -334,7 +342,7 @@ def run_gpu(args, cfg):
         achieved = fl / (launch_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[pk_key], "unit": "TFLOP/s",
                 "frac": achieved / peaks[pk_key]}
-        value = world * fl / (ms_per_step / 1e3) / 1e12
+        value = job_throughput(fl, world, total_ms, args.steps) / 1e12
         unit = "TFLOP/s"
         e2e_value = world * fl / (e2e_ms / 1e3) / 1e12
     roof["peak_source"] = f"{peak_src}:" + ("hbm_gbs" if decode_like else pk_key)

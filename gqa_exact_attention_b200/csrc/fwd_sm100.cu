@@ -63,7 +63,7 @@ struct FwdCfg {
     static_assert(!kEpilogueWG || (kRegsEpilogue >= 64 && kRegsEpilogue % 8 == 0),
                   "epilogue registers");
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
-    static constexpr int kNumBars = 2 * kSlots + 7 * NT + 1;
+    static constexpr int kNumBars = 2 * kSlots + 8 * NT + 1;
     static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + NT * kTileBytes +
                                       kSlots * kTileBytes + 8 * kNumBars + kStatsBytes + 16;
@@ -272,8 +272,12 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
     auto p_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 3 * NT + t); };
     auto o_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 4 * NT + t); };
     auto o_empty = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 5 * NT + t); };
-    auto st_full = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 6 * NT + t); };
-    const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 7 * NT);
+    // One barrier per statistics buffer: the softmax may post a unit's statistics before
+    // the epilogue has waited for the previous unit's (a one-block unit's S needs nothing
+    // from the epilogue), and a parity wait must never fall two phases behind.  Per buffer,
+    // the next post needs the epilogue to have released O_t of the unit before.
+    auto st_full = [&](int t, uint32_t buf) { return bar0 + 8u * (2 * C::kSlots + 6 * NT + 2 * t + buf); };
+    const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 8 * NT);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -291,7 +295,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
             mbar_init(p_full(t), 128);
             mbar_init(o_full(t), 1);
             mbar_init(o_empty(t), 128);
-            mbar_init(st_full(t), 128);
+            mbar_init(st_full(t, 0), 128);
+            mbar_init(st_full(t, 1), 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0u;
@@ -556,8 +561,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 }
                 if (!ok) break;
                 if constexpr (C::kEpilogueWG) {
+                    mbar_arrive(st_full(t, stn & 1u));
                     ++stn;
-                    mbar_arrive(st_full(t));
                 } else {
                     ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), sn_o & 1u, abort_flag, p));
                     if (!ok) break;
@@ -683,8 +688,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 float* st = stats + ((stn & 1u) * NT + t) * 256;
                 st[row] = m;
                 st[128 + row] = l;
+                mbar_arrive(st_full(t, stn & 1u));
                 ++stn;
-                mbar_arrive(st_full(t));
             } else {
                 ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), sn_o & 1u, abort_flag, p));
                 if (!ok) break;
@@ -711,7 +716,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 const bool idle = __all_sync(0xffffffffu, !rm.ok);
                 float m = -INFINITY, l = 0.f;
                 if (has) {
-                    ok = __all_sync(0xffffffffu, wait_bounded(st_full(t), stn[t] & 1u, abort_flag, p));
+                    ok = __all_sync(0xffffffffu, wait_bounded(st_full(t, stn[t] & 1u), (stn[t] >> 1) & 1u,
+                                                              abort_flag, p));
                     if (!ok) break;
                     const float* st = stats + ((stn[t] & 1u) * NT + t) * 256;
                     m = st[row];

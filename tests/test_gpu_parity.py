@@ -109,3 +109,16 @@ def test_odd_sq77_sk4096(d, hk):
     o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(d), 0)
     out, lse = run(q, k, v, 0)
     P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"Sq77 d{d} hk{hk}")
+
+
+# --- many units per persistent CTA with causal split-KV: units whose tiles have zero or
+#     one key block let a softmax warpgroup run ahead of the epilogue; full oracle
+@pytest.mark.parametrize("shp,splits", [((8, 2048, 2048, 4, 2, 128), 3),
+                                         ((16, 1024, 1024, 4, 2, 128), 3),
+                                         ((8, 2048, 2048, 4, 2, 64), 4)])
+def test_many_units_causal_splits(shp, splits):
+    seed = 3300 + splits
+    q, k, v = P.device_inputs(seed, *shp)
+    o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(shp[-1]), 1)
+    out, lse = run(q, k, v, 1, 0, splits)
+    P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"{shp} s{splits}")
