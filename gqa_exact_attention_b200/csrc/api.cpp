@@ -151,6 +151,21 @@ bool encode_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, in
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 output [Bs, S, H, d] (Bs = B, or splits * B for the partials) as a 4-D map
+// (d, H, S, Bs) for TMA stores: 128-byte swizzle, box (32, box_h, box_s, 1).
+bool encode_out(CUtensorMap* m, const void* ptr, int Bs, int S, int H, int d, int box_h,
+                int box_s) {
+    EncodeTiled enc = get_encode_tiled();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)Bs};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)S * H * d * 4};
+    cuuint32_t box[4] = {32, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceInfo {
     int sms = 0;
     int ok = 0;  // 1: sm_100
@@ -298,6 +313,12 @@ gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out,
         p.o_part = static_cast<float*>(ws);
         p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
     }
+    if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
+                    pl.splits > 1 ? pl.splits * B : B, Sq, Hq, d, pl.pack ? g : 1,
+                    pl.pack ? pl.pos_per_tile : kBlockM)) {
+        if (ws) cudaFreeAsync(ws, stream);
+        return GQA_ERR_CUDA;
+    }
 
     const int slots = info.sms * gqa::fwd_ctas_per_sm(d, pl.nt);
     const int grid = (int)(pl.units < slots ? pl.units : slots);
@@ -395,6 +416,10 @@ gqa_status fwd_with_scratch(const void* q, const void* k, const void* v, float* 
         p.o_part = static_cast<float*>(scratch);
         p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
     }
+    if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
+                    pl.splits > 1 ? pl.splits * B : B, Sq, Hq, d, pl.pack ? g : 1,
+                    pl.pack ? pl.pos_per_tile : kBlockM))
+        return GQA_ERR_CUDA;
     const int slots = info.sms * fwd_ctas_per_sm(d, pl.nt);
     const int grid = (int)(pl.units < slots ? pl.units : slots);
     if (launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) return GQA_ERR_CUDA;

@@ -18,10 +18,12 @@ struct FwdParams {
     CUtensorMap tm_q;  // q as 4-D (d, Hq, Sq, B); box (64, g or 1, positions, 1)
     CUtensorMap tm_k;  // k as 4-D (d, Hk, Sk, B); box (64, 1, 128, 1)
     CUtensorMap tm_v;  // v likewise
+    CUtensorMap tm_o;  // fp32 output for TMA stores: out as (d, Hq, Sq, B), or the split
+                       // partials as (d, Hq, Sq, splits*B); box (32, g or 1, positions, 1)
 
     float* out;       // [B, Sq, Hq, d]       (num_splits == 1)
     float* lse;       // [B, Hq, Sq]          (num_splits == 1)
-    float* o_part;    // [splits, B, Hq, Sq, d] (num_splits > 1)
+    float* o_part;    // [splits, B, Sq, Hq, d] (num_splits > 1)
     float* lse_part;  // [splits, B, Hq, Sq]    (num_splits > 1)
 
     int B, Sq, Sk, Hq, Hk;

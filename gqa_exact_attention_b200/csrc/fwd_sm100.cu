@@ -65,8 +65,11 @@ struct FwdCfg {
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
     static constexpr int kNumBars = 2 * kSlots + 8 * NT + 1;
     static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
+    // epilogue staging for TMA stores: 128 rows x 32 fp32 (128 B, swizzled) per chunk
+    static constexpr int kOStageBytes = kEpilogueWG ? 128 * 128 : 0;
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + NT * kTileBytes +
-                                      kSlots * kTileBytes + 8 * kNumBars + kStatsBytes + 16;
+                                      kSlots * kTileBytes + kOStageBytes + 8 * kNumBars +
+                                      kStatsBytes + 16;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, HD, true);
@@ -185,9 +188,9 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, c
         orow = p.out + (((size_t)b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
         lrow = p.lse + ((size_t)b * p.Hq + rm.head) * p.Sq + rm.pos;
     } else {
-        const size_t r = (((size_t)split * p.B + b) * p.Hq + rm.head) * p.Sq + rm.pos;
-        orow = p.o_part + r * HD;
-        lrow = p.lse_part + r;
+        const size_t sb = (size_t)split * p.B + b;
+        orow = p.o_part + ((sb * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
+        lrow = p.lse_part + (sb * p.Hq + rm.head) * p.Sq + rm.pos;
     }
 #pragma unroll
     for (int ch = 0; ch < HD / 32; ++ch) {
@@ -258,7 +261,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
 
     const uint32_t sQ = base;
     const uint32_t sKV = base + NT * C::kTileBytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NT * C::kTileBytes + C::kSlots * C::kTileBytes);
+    const uint32_t sO = sKV + C::kSlots * C::kTileBytes;  // 1024-aligned staging (NT == 2)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NT * C::kTileBytes + C::kSlots * C::kTileBytes +
+                                                 C::kOStageBytes);
     float* stats = reinterpret_cast<float*>(bars + C::kNumBars);  // [2][NT][2][128]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(stats) + C::kStatsBytes);
     volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -700,10 +705,16 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
         }
     } else if constexpr (C::kEpilogueWG) {
         // ------------------------------------------------------------ epilogue
+        // O / l goes out through a swizzled shared-memory stage and TMA tensor stores, a
+        // 32-column chunk at a time, so every global write is a full line; LSE is stored
+        // directly.
         if constexpr (C::kRegsEpilogue < C::kLaunchRegs) regs_dec<C::kRegsEpilogue>();
         if constexpr (C::kRegsEpilogue > C::kLaunchRegs) regs_inc<C::kRegsEpilogue>();
+        constexpr uint32_t kEpiBar = 1;  // named barrier of the four epilogue warps
+        constexpr float kLn2 = 0.69314718055994530942f;
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
+        const bool issuer = (threadIdx.x == (1 + NT) * 128);
         uint32_t on[NT] = {}, stn[NT] = {};
         bool ok = true;
         for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -711,6 +722,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 if (!ok) break;
+                if (g.pos0[t] >= p.Sq) continue;  // a tile wholly past the query axis (uniform)
                 const RowMap rm = row_map(p, g.pos0[t], g.hg, row);
                 const bool has = g.n[t] > 0;
                 const bool idle = __all_sync(0xffffffffu, !rm.ok);
@@ -718,20 +730,70 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 if (has) {
                     ok = __all_sync(0xffffffffu, wait_bounded(st_full(t, stn[t] & 1u), (stn[t] >> 1) & 1u,
                                                               abort_flag, p));
-                    if (!ok) break;
-                    const float* st = stats + ((stn[t] & 1u) * NT + t) * 256;
-                    m = st[row];
-                    l = st[128 + row];
-                    ++stn[t];
-                    ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), on[t] & 1u, abort_flag, p));
-                    if (!ok) break;
-                    ++on[t];
-                    tc_fence_after();
+                    if (ok) {
+                        const float* st = stats + ((stn[t] & 1u) * NT + t) * 256;
+                        m = st[row];
+                        l = st[128 + row];
+                        ++stn[t];
+                        ok = __all_sync(0xffffffffu, wait_bounded(o_full(t), on[t] & 1u, abort_flag, p));
+                        ++on[t];
+                    }
                 }
+                // one decision for the whole warpgroup before its named barriers
+                ok = named_bar_and(kEpiBar, 128, ok);
+                if (!ok) break;
+                tc_fence_after();
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
                 const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
-                write_row<HD>(p, o_addr, rm, g.b, g.split, has, idle, m, l, o_empty(t));
+                const int hcoord = p.pack ? g.hg * p.g : g.hg;
+                const int bcoord = p.num_splits == 1 ? g.b : g.split * p.B + g.b;
+#pragma unroll
+                for (int ch = 0; ch < HD / 32; ++ch) {
+                    uint32_t r[32];
+                    if (has && !idle) {
+                        tmem_ld32(o_addr + ch * 32, r);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = 0u;
+                    }
+                    if (has && ch == HD / 32 - 1) {
+                        // O_t is in registers: the next unit's PV may overwrite it
+                        tc_fence_before();
+                        mbar_arrive(o_empty(t));
+                    }
+                    // the stage is free once the previous store has read it
+                    if (issuer) bulk_wait_read_all();
+                    named_bar_sync(kEpiBar, 128);
+                    const uint32_t dst = sO + row * 128;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t a = dst + ((uint32_t)(i ^ (row & 7)) << 4);
+                        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                                     "f"(__uint_as_float(r[4 * i + 0]) * inv_l),
+                                     "f"(__uint_as_float(r[4 * i + 1]) * inv_l),
+                                     "f"(__uint_as_float(r[4 * i + 2]) * inv_l),
+                                     "f"(__uint_as_float(r[4 * i + 3]) * inv_l)
+                                     : "memory");
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(kEpiBar, 128);
+                    if (issuer) {
+                        tma_store_4d(&p.tm_o, sO, ch * 32, hcoord, g.pos0[t], bcoord);
+                        bulk_commit_group();
+                    }
+                }
+                if (rm.ok) {
+                    if (p.num_splits == 1)
+                        p.lse[((size_t)g.b * p.Hq + rm.head) * p.Sq + rm.pos] = lse_v;
+                    else
+                        p.lse_part[(((size_t)g.split * p.B + g.b) * p.Hq + rm.head) * p.Sq + rm.pos] = lse_v;
+                }
             }
         }
+        if (issuer) bulk_wait_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -765,10 +827,14 @@ __global__ void __launch_bounds__(256) gqa_combine_kernel(const CombineParams p)
         float acc[kPer];
 #pragma unroll
         for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+        // r = (b * Hq + h) * Sq + i; partials are [split, B, Sq, Hq, d]
+        const long long ii = r % p.Sq;
+        const long long hh = (r / p.Sq) % p.Hq;
+        const long long bb = r / ((long long)p.Sq * p.Hq);
         for (int s = 0; s < p.num_splits; ++s) {
             const float ws = __shfl_sync(0xffffffffu, w, s);
             if (ws == 0.f) continue;
-            const float* src = p.o_part + ((long long)s * rows + r) * HD + lane * kPer;
+            const float* src = p.o_part + ((((long long)s * p.B + bb) * p.Sq + ii) * p.Hq + hh) * HD + lane * kPer;
             if constexpr (kPer == 4) {
                 const float4 v = *reinterpret_cast<const float4*>(src);
                 acc[0] += ws * v.x;
