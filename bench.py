@@ -418,6 +418,66 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Kernel-only timings over the batch-size sweep (B 16..256, causal and not, every
+    pack/split variant plus the heuristic's choice) or the decode grid (Sk 2K/8K/32K,
+    B 32/128/256, splits 1/2/4/8 plus the heuristic's).  One JSON line per case; not the
+    benchmark contract's line."""
+    import torch
+
+    import gqa_exact_attention_b200 as G
+    import inputs
+    torch.cuda.set_device(0)
+    G.load()
+    stream = torch.cuda.current_stream()
+    peaks, _ = load_peaks()
+    if args.sweep == "prefill":
+        cases = [(B, 2048, 2048, c, pk, sp) for B in (16, 32, 64, 128, 256) for c in (1, 0)
+                 for (pk, sp) in [(-1, 0), (0, 1), (1, 1), (0, 2), (1, 2), (0, 4), (1, 4)]]
+    else:
+        cases = [(B, 1, Sk, 0, pk, sp) for Sk in (2048, 8192, 32768) for B in (32, 128, 256)
+                 for (pk, sp) in [(-1, 0), (1, 1), (1, 2), (1, 4), (1, 8)]]
+    cur = None
+    for (B, Sq, Sk, causal, pk, sp) in cases:
+        Hq, Hk, d = 32, 8, 128
+        if cur != (B, Sq, Sk):
+            q = k = v = out = lse = None
+            torch.cuda.empty_cache()
+            q = inputs.device_tensor(1001, inputs.TID_Q, (B, Sq, Hq, d))
+            k = inputs.device_tensor(1001, inputs.TID_K, (B, Sk, Hk, d))
+            v = inputs.device_tensor(1001, inputs.TID_V, (B, Sk, Hk, d))
+            out = torch.empty((B, Sq, Hq, d), dtype=torch.float32, device="cuda")
+            lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
+            cur = (B, Sq, Sk)
+        rp, rs = G.gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, causal) if (pk < 0 and sp <= 0) else (pk, sp)
+
+        def step():
+            G.gqa_attn_fwd(q, k, v, out=out, lse=lse, causal=causal, pack_gqa=rp,
+                           num_splits=rs, stream=stream)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        fl = flops(B, Sq, Sk, Hq, d, causal)
+        by = hbm_bytes(B, Sq, Sk, Hq, Hk, d)
+        line = {"sweep": args.sweep, "B": B, "Sq": Sq, "Sk": Sk, "causal": bool(causal),
+                "pack_gqa": rp, "num_splits": rs, "heuristic": pk < 0 and sp <= 0,
+                "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1),
+                "hbm_gbs": round(by / ms / 1e6, 1),
+                "tokens_per_s": round(B * (Sq if Sq > 1 else 1) / ms * 1e3, 1)}
+        if args.sweep == "prefill":
+            line["frac_of_measured_bf16"] = round(fl / ms / 1e9 / peaks["bf16_tflops"], 3)
+        else:
+            line["frac_of_measured_hbm"] = round(by / ms / 1e6 / peaks["hbm_gbs"], 3)
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,6 +495,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", choices=["prefill", "decode"], default=None,
+                    help="print one line per configuration of the batch sweep or decode grid")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -449,6 +511,8 @@ def main():
                   if in_bytes > 126e6 else f"inputs {in_bytes / 1e6:.1f} MB, L2-resident")}
     if args.impl == "reference":
         run_reference(args, cfg)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_gpu(args, cfg)
 

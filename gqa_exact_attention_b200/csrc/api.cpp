@@ -80,17 +80,21 @@ Plan make_plan(int B, int Sq, int Sk, int Hq, int Hk, int pack) {
 }
 
 // Split count minimising the modelled time: waves(s) x (key blocks per split + a fixed
-// per-unit cost of about one block: Q load, pipeline fill, epilogue).  A persistent CTA
-// per SM takes units in a static stride, so a partial last wave costs a whole unit time.
+// per-unit cost).  A persistent CTA per SM slot takes units in a static stride, so a
+// partial last wave costs a whole unit time.  The fixed cost (Q load, pipeline fill,
+// epilogue, and the partials' write and combine) was fitted to B200 measurements of
+// the decode grid (Sk 2K-32K, B 32-256): about four key blocks' worth; a split must
+// also buy at least 5 %, since the combine adds a launch.
 int choose_splits(const Plan& pl, int d, int num_sms) {
     const long long slots = (long long)num_sms * gqa::fwd_ctas_per_sm(d, pl.nt);
     const int smax = pl.kv_blocks < kMaxSplits ? pl.kv_blocks : kMaxSplits;
+    constexpr double kUnitCost = 4.0;
     int best = 1;
     double best_t = 0.0;
     for (int s = 1; s <= smax; ++s) {
         const long long waves = (pl.units * s + slots - 1) / slots;
-        const double t = (double)waves * ((double)pl.kv_blocks / s + 1.0);
-        if (s == 1 || t < best_t * 0.97) {  // a split must buy at least 3 %
+        const double t = (double)waves * ((double)pl.kv_blocks / s + kUnitCost);
+        if (s == 1 || t < best_t * 0.95) {
             best = s;
             best_t = t;
         }
@@ -204,6 +208,41 @@ int batch_window(int B, int Sk, int Hk, int d) {
     return w < B ? w : B;
 }
 
+void set_unit_divisors(gqa::FwdParams* p, int B) {
+    const int per_batch = p->n_hg * p->n_mt * p->num_splits;
+    p->div_window = gqa::make_fastdiv((uint32_t)(p->batch_window * per_batch));
+    p->div_splits = gqa::make_fastdiv((uint32_t)p->num_splits);
+    p->div_hg = gqa::make_fastdiv((uint32_t)p->n_hg);
+    p->div_bw = gqa::make_fastdiv((uint32_t)p->batch_window);
+    const int last = B % p->batch_window;
+    p->div_bw_last = gqa::make_fastdiv((uint32_t)(last == 0 ? p->batch_window : last));
+}
+
+// Split-KV scratch comes from a library-owned stream-ordered pool per device that keeps
+// its memory (release threshold = max), so a host synchronisation does not hand the
+// memory back to the driver and make the next call map it again.
+cudaMemPool_t workspace_pool(int dev) {
+    static cudaMemPool_t pools[64] = {};
+    static std::mutex mu;
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (pools[dev] == nullptr) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        uint64_t keep = ~0ull;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 long long timeout_ns() {
@@ -295,6 +334,7 @@ gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out,
     p.n_mt = pl.n_mt;
     p.n_units = (int)pl.units;
     p.batch_window = batch_window(B, Sk, Hk, d);
+    set_unit_divisors(&p, B);
     p.kv_blocks = pl.kv_blocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.div_g = gqa::make_fastdiv((uint32_t)g);
@@ -306,7 +346,8 @@ gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out,
         const size_t rows = (size_t)B * Hq * Sq;
         const size_t bytes = (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
         if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
-        if (cudaMallocAsync(&ws, bytes, stream) != cudaSuccess) {
+        cudaMemPool_t pool = workspace_pool(dev);
+        if (pool == nullptr || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess) {
             cudaGetLastError();
             return GQA_ERR_ALLOC;
         }
@@ -407,6 +448,7 @@ gqa_status fwd_with_scratch(const void* q, const void* k, const void* v, float* 
     p.n_mt = pl.n_mt;
     p.n_units = (int)pl.units;
     p.batch_window = batch_window(B, Sk, Hk, d);
+    set_unit_divisors(&p, B);
     p.kv_blocks = pl.kv_blocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.div_g = make_fastdiv((uint32_t)g);

@@ -40,6 +40,9 @@ struct FwdParams {
     int kv_blocks;     // ceil(Sk / 128)
     float scale_log2;  // scale * log2(e)
     FastDiv div_g;     // row -> (position, head-in-group) for packed tiles
+    // unit index decomposition (see unit_geom): window size, splits, heads-or-groups,
+    // batches per full window and in the last (possibly partial) window
+    FastDiv div_window, div_splits, div_hg, div_bw, div_bw_last;
     unsigned int* status;  // status word for bounded-wait timeouts (NULL: the library's own)
     long long timeout_ns;  // limit of each in-kernel wait
 };

@@ -103,19 +103,20 @@ struct UnitGeom {
 // keeps every K/V block's readers close together in time.
 template <int NT>
 __device__ __forceinline__ UnitGeom<NT> unit_geom(int u, const FwdParams& p) {
+    // all divisions by run-time sizes are multiply-shift (FastDiv), computed on the host
     UnitGeom<NT> g;
-    const int per_batch = p.n_hg * p.n_mt * p.num_splits;
-    const int w = u / (p.batch_window * per_batch);
-    int r = u - w * p.batch_window * per_batch;
-    const int b0 = w * p.batch_window;
-    const int nb = min(p.batch_window, p.B - b0);
-    g.split = r % p.num_splits;
-    r /= p.num_splits;
-    g.hg = r % p.n_hg;
-    r /= p.n_hg;
-    g.b = b0 + r % nb;
-    const int mt = p.n_mt - 1 - r / nb;
-    g.kvh = p.pack ? g.hg : g.hg / p.g;
+    uint32_t w, r, q, rem;
+    fastdivmod((uint32_t)u, p.div_window, w, r);
+    const int b0 = (int)w * p.batch_window;
+    const bool last = b0 + p.batch_window > p.B;
+    fastdivmod(r, p.div_splits, q, rem);
+    g.split = (int)rem;
+    fastdivmod(q, p.div_hg, r, rem);
+    g.hg = (int)rem;
+    fastdivmod(r, last ? p.div_bw_last : p.div_bw, q, rem);
+    g.b = b0 + (int)rem;
+    const int mt = p.n_mt - 1 - (int)q;
+    g.kvh = p.pack ? g.hg : (int)fastdiv((uint32_t)g.hg, p.div_g);
     int kb_end[NT];
     int kb_union = 0;
 #pragma unroll

@@ -85,9 +85,10 @@ typedef enum {
  *   pack_gqa    -1 = chosen by gqa_attn_choose, 0 = one q-head per tile, 1 = packed.
  *   num_splits  0 = chosen by gqa_attn_choose, >= 1 = that many key ranges.  Clamped to
  *               the number of 128-key blocks and to 16.  With more than one split the
- *               library allocates stream-ordered scratch (cudaMallocAsync on `stream`,
- *               freed with cudaFreeAsync after the combine on the same stream) of
- *               gqa_attn_workspace_bytes(...) bytes.
+ *               library allocates stream-ordered scratch of gqa_attn_workspace_bytes(...)
+ *               bytes from its own per-device memory pool (cudaMallocFromPoolAsync on
+ *               `stream`, freed with cudaFreeAsync after the combine on the same stream;
+ *               the pool keeps freed memory for reuse until the process exits).
  *
  * Errors: argument errors return before anything is launched or written.  Launch
  * errors return GQA_ERR_CUDA.  A device-side bounded-wait timeout (which should not

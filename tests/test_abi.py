@@ -100,10 +100,13 @@ def test_heuristic_splits():
     assert G.gqa_attn_choose(64, 2048, 2048, 32, 8, 128, 1)[1] == 1
     assert G.gqa_attn_choose(16, 2048, 2048, 32, 8, 128, 0)[1] == 1
     # small decode batch -> split the key axis, bounded by the key blocks and 16
-    pk, ns = G.gqa_attn_choose(32, 1, 8192, 32, 8, 128, 0)
-    assert 2 <= ns <= 8
-    # large decode batch: 256 x 8 units already fill the SMs
+    # a decode batch whose (batch, kv-head) units nearly fill the SM slots: no split
+    # (measured on B200: splitting B=32, Sk=8192 costs more than it spreads)
+    assert G.gqa_attn_choose(32, 1, 8192, 32, 8, 128, 0)[1] == 1
     assert G.gqa_attn_choose(256, 1, 8192, 32, 8, 128, 0)[1] == 1
+    # a small decode batch: split the key axis
+    pk, ns = G.gqa_attn_choose(4, 1, 8192, 32, 8, 128, 0)
+    assert 2 <= ns <= 16
     assert G.gqa_attn_choose(1, 1, 256, 32, 8, 128, 0)[1] <= 2
     assert G.gqa_attn_choose(1, 1, 1 << 20, 32, 8, 128, 0)[1] <= 16
 
