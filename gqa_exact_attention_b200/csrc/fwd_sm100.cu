@@ -597,39 +597,14 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 tmem_wait_ld();
                 const int lim = kmax - (g.kb_lo + it) * kBlockN;  // keys [0, lim) allowed
                 const bool masked = lim < kBlockN;
+                // disallowed keys (j >= lim) take the fill value, which drops them out of
+                // the extremum below
                 if (masked) {
 #pragma unroll
                     for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : fill;
                 }
-                // P = 2^(c*s - m) against the current reference max m, computed before
-                // the block's own max is known (that max only decides whether m has to
-                // move, which is rare after a row's first block).  First half: 64 keys.
-                float neg_m = (m == kNegInf) ? 0.f : -m;
-                float ls0 = 0.f, ls1 = 0.f;
-                // exponentials of keys [32*ch0, 32*ch1), packed to bf16 and stored over S
-                auto exp_range = [&](int ch0, int ch1) {
-#pragma unroll
-                    for (int ch = ch0; ch < ch1; ++ch) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int j = ch * 32 + 2 * i;
-                            float x0, x1;
-                            fma2(s[j], s[j + 1], c, c, neg_m, neg_m, x0, x1);
-                            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                            if (masked) {
-                                p0 = (j < lim) ? p0 : 0.f;
-                                p1 = (j + 1 < lim) ? p1 : 0.f;
-                            }
-                            add2(ls0, ls1, p0, p1, ls0, ls1);
-                            pk[i] = pack_bf16x2(p0, p1);
-                        }
-                        tmem_st16(s_addr + ch * 16, pk);
-                    }
-                };
-                if (it > 0) exp_range(0, 2);
-                // extremum of the raw scores (max for c >= 0, min for c < 0), times c:
-                // eight chains of three-input max/min
+                // extremum of the raw scores over the allowed keys (max for c >= 0, min
+                // for c < 0), times c: eight chains of three-input max/min
                 float e[8];
                 if (c >= 0.f) {
 #pragma unroll
@@ -659,16 +634,34 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                     alpha = (m == kNegInf) ? 0.f : ex2_approx(m - mx);
                     l *= alpha;
                     m = mx;
-                    neg_m = -m;
                 }
-                if (it == 0 || __any_sync(0xffffffffu, grow)) {
-                    // (re)compute the first half against the moved reference max
-                    ls0 = 0.f;
-                    ls1 = 0.f;
-                    exp_range(0, 2);
-                }
-                // O rescale before the first P.V of this block: PV of the previous block
-                // is complete, because this block's S was issued after it.
+                // P = 2^(c*s - m) as bf16, written over S in TMEM (S is in registers).  A
+                // disallowed key gets the exponent -inf, i.e. p = 0, for any sign of c.
+                const float neg_m = (m == kNegInf) ? 0.f : -m;
+                float ls0 = 0.f, ls1 = 0.f;
+                auto exp_range = [&](int ch0, int ch1) {
+#pragma unroll
+                    for (int ch = ch0; ch < ch1; ++ch) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int j = ch * 32 + 2 * i;
+                            float x0, x1;
+                            fma2(s[j], s[j + 1], c, c, neg_m, neg_m, x0, x1);
+                            if (masked) {
+                                x0 = (j < lim) ? x0 : kNegInf;
+                                x1 = (j + 1 < lim) ? x1 : kNegInf;
+                            }
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            add2(ls0, ls1, p0, p1, ls0, ls1);
+                            pk[i] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st16(s_addr + ch * 16, pk);
+                    }
+                };
+                exp_range(0, 2);
+                // O rescale: PV of the previous block is complete, because this block's S
+                // was issued after it.
                 if (it > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
                     for (int ch = 0; ch < HD / 32; ++ch) {
