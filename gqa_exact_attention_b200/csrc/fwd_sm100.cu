@@ -54,8 +54,8 @@ struct FwdCfg {
     // warpgroups x launch regs, so every increase is covered by the decreases (each SM
     // sub-partition holds one warp of each warpgroup)
     static constexpr int kLaunchRegs = ((65536 / (kThreads * kCtasPerSm)) / 8) * 8;
-    static constexpr int kRegsLoad = NT == 2 ? 96 : 56;
-    static constexpr int kRegsSoftmax = NT == 2 ? 168 : 200;
+    static constexpr int kRegsLoad = NT == 2 ? 104 : 80;
+    static constexpr int kRegsSoftmax = NT == 2 ? 168 : 176;
     static constexpr int kRegsEpilogue =
         kEpilogueWG ? kWarpgroups * kLaunchRegs - kRegsLoad - NT * kRegsSoftmax : 0;
     static_assert(kRegsLoad + NT * kRegsSoftmax + kRegsEpilogue == kWarpgroups * kLaunchRegs,
@@ -331,26 +331,30 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
             uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
             uint32_t qn[NT] = {};  // Q loads issued per tile
             bool ok = true;
+            // Q_t of a unit, once the previous unit's last S_t has read the buffer
+            auto load_q = [&](const UnitGeom<NT>& g, int t) {
+                if (g.n[t] == 0 || !ok) return;
+                if (qn[t] > 0)
+                    ok = __all_sync(0xffffffffu, wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p));
+                if (!ok) return;
+                if (elect_one()) {
+                    const int rows = p.pack ? p.rows_valid : kBlockM;
+                    mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
+                    const int hcoord = p.pack ? g.hg * p.g : g.hg;
+#pragma unroll
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
+                                    q_full(t), c * 64, hcoord, g.pos0[t], g.b);
+                }
+                __syncwarp();
+                ++qn[t];
+            };
+            // Load order per unit: Q_0, K_0, Q_1.., V_0, K_1, V_1, ...  The MMA warp may
+            // issue a unit's first S_0 while the unit before still runs on tile 1, so K_0
+            // must not queue behind Q_1 (which waits for that unit's last S_1).
             for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
                 const UnitGeom<NT> g = unit_geom<NT>(u, p);
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (g.n[t] == 0 || !ok) continue;
-                    if (qn[t] > 0)
-                        ok = __all_sync(0xffffffffu, wait_bounded(q_empty(t), (qn[t] - 1) & 1u, abort_flag, p));
-                    if (!ok) break;
-                    if (elect_one()) {
-                        const int rows = p.pack ? p.rows_valid : kBlockM;
-                        mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
-                        const int hcoord = p.pack ? g.hg * p.g : g.hg;
-#pragma unroll
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
-                                        q_full(t), c * 64, hcoord, g.pos0[t], g.b);
-                    }
-                    __syncwarp();
-                    ++qn[t];
-                }
+                load_q(g, 0);
                 for (int it = 0; it < g.nblk && ok; ++it) {
                     const int kpos = (g.kb_lo + it) * kBlockN;
 #pragma unroll
@@ -369,6 +373,10 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                         }
                         __syncwarp();
                         ++ld;
+                        if (it == 0 && w == 0) {
+#pragma unroll
+                            for (int t = 1; t < NT; ++t) load_q(g, t);
+                        }
                     }
                 }
             }
@@ -436,17 +444,31 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p));
             };
 
+            // A tile that finishes its unit starts the next unit at once: its first S_t is
+            // issued right after its last PV_t (the tensor pipe runs MMAs in issue order,
+            // so S_t may overwrite the P_t that PV_t reads), instead of after every tile's
+            // last PV.  early[t]: the current unit's first S_t was issued that way.
+            bool early[NT] = {};
             for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
                 const UnitGeom<NT> g = unit_geom<NT>(u, p);
+                // key blocks per tile of the next unit (0 when there is none)
+                int n_next[NT] = {};
+                if (u + (int)gridDim.x < p.n_units) {
+                    const UnitGeom<NT> gn = unit_geom<NT>(u + (int)gridDim.x, p);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) n_next[t] = gn.n[t];
+                }
+                bool early_next[NT] = {};
                 if (g.nblk == 0) continue;
-                // first key block: S_t for every tile that has keys
+                // first key block: S_t for every tile that has keys (and was not started)
+                const uint32_t ld_unit = ld;  // ring index of this unit's first K block
                 int slot_k = ld % C::kSlots;
                 ok = wait(kv_full(slot_k), (ld / C::kSlots) & 1u);
                 if (!ok) break;
                 ++ld;
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
-                    if (g.n[t] == 0 || !ok) continue;
+                    if (g.n[t] == 0 || early[t] || !ok) continue;
                     ok = wait(q_full(t), qn[t] & 1u);
                     if (!ok) break;
                     ++qn[t];
@@ -516,12 +538,31 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                             p_ready = has_next_tile && probed;
                             commit(o_full(t));
                             ++on[t];
+                            // The next unit's K_0 sits at ring index ld_unit + 2 nblk.  Taking
+                            // it now is safe when the ring entry it replaces was consumed and
+                            // released by an earlier iteration (or the prologue): then its
+                            // barrier phase is current and the producer is not blocked on
+                            // anything issued later.
+                            if (n_next[t] > 0 && 2 * (g.nblk - it) <= C::kSlots) {
+                                const uint32_t kq = ld_unit + 2u * (uint32_t)g.nblk;
+                                ok = wait(kv_full(kq % C::kSlots), (kq / C::kSlots) & 1u);
+                                if (ok) ok = wait(q_full(t), qn[t] & 1u);
+                                if (!ok) break;
+                                ++qn[t];
+                                tc_fence_after();
+                                issue_s(t, kq % C::kSlots, 0u, 0u);
+                                commit(s_full(t));
+                                if (n_next[t] == 1) commit(q_empty(t));
+                                early_next[t] = true;
+                            }
                         }
                     }
                     if (!ok) break;
                     commit(kv_empty(slot_v));
                     if (next) commit(kv_empty(slot_n));
                 }
+#pragma unroll
+                for (int t = 0; t < NT; ++t) early[t] = early_next[t];
             }
             // every MMA issued so far must be complete before TMEM is released
             commit(mma_done);
