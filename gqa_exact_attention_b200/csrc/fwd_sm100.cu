@@ -22,10 +22,15 @@
 #include <cuda_runtime.h>
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "fwd_params.h"
 #include "launch.h"
 #include "ptx_sm100.cuh"
+
+#ifndef GQA_EXP_POLY_PAIRS
+#define GQA_EXP_POLY_PAIRS 4
+#endif
 
 namespace gqa {
 
@@ -62,6 +67,9 @@ struct FwdCfg {
                   "register split must add up to the launch allocation");
     static_assert(!kEpilogueWG || (kRegsEpilogue >= 64 && kRegsEpilogue % 8 == 0),
                   "epilogue registers");
+    // of each 16 exponential pairs of a 32-key chunk, this many take the polynomial (unmasked
+    // blocks only); the rest use the special-function unit
+    static constexpr int kPolyPairs = GQA_EXP_POLY_PAIRS;
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
     static constexpr int kNumBars = 2 * kSlots + 8 * NT + 1;
     static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
@@ -76,6 +84,31 @@ struct FwdCfg {
     __host__ __device__ static constexpr int s_col(int t) { return t * 128; }
     __host__ __device__ static constexpr int o_col(int t) { return NT * 128 + t * HD; }
 };
+
+// 2^x on the FMA and integer pipes, for a share of the exponentials so that they do not
+// all queue on the special-function unit.  Cody-Waite reduction x = j + f with j = rint(x)
+// (the 1.5 * 2^23 rounding constant puts j in the low mantissa bits of t), then
+// 2^f ~ 1 + f (c1 + f (c2 + f c3)) on [-1/2, 1/2]: a degree-3 fit minimising the relative
+// error with the constant term held at 1, max relative error 1.02e-4 (the bf16 rounding
+// of P is 2^-9 = 1.95e-3); 2^j is added to the exponent field.  x is clamped at -126 so the
+// exponent cannot underflow (the result there is 2^-126 instead of a smaller number);
+// inputs are at most 8 (the deferred-rescale bound), far below overflow.  Only for finite x:
+// masked keys keep the exact zero of the special-function path.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+    constexpr float c1 = 0.6932829022407532f, c2 = 0.24221095442771912f, c3 = 0.055008936673402786f;
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float t0, t1, r0, r1, f0, f1, q0, q1;
+    add2(x0, x1, kRound, kRound, t0, t1);
+    add2(t0, t1, -kRound, -kRound, r0, r1);
+    add2(x0, x1, -r0, -r1, f0, f1);
+    fma2(f0, f1, c3, c3, c2, c2, q0, q1);
+    fma2(q0, q1, f0, f1, c1, c1, q0, q1);
+    fma2(q0, q1, f0, f1, 1.f, 1.f, q0, q1);
+    y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
 
 template <uint32_t R>
 __device__ __forceinline__ void regs_inc() {
@@ -637,35 +670,57 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 }
                 tmem_wait_ld();
                 const int lim = kmax - (g.kb_lo + it) * kBlockN;  // keys [0, lim) allowed
-                const bool masked = lim < kBlockN;
-                // disallowed keys (j >= lim) take the fill value, which drops them out of
-                // the extremum below
-                if (masked) {
+                // Warp-uniform view of the mask, per 32-key chunk: every key allowed for all
+                // 32 rows of the warp (full), none allowed for any of them (empty), or in
+                // between.  The branches on it are uniform, as the warp-collective tcgen05.st
+                // in the exponential loop requires.  Unmasked blocks skip all of it.
+                const int lim_lo = __reduce_min_sync(0xffffffffu, lim);
+                const int lim_hi = __reduce_max_sync(0xffffffffu, lim);
+                const bool masked = lim_lo < kBlockN;
+                auto chunk_empty = [&](int ch) { return ch * 32 >= lim_hi; };
+                auto chunk_full = [&](int ch) { return ch * 32 + 32 <= lim_lo; };
+                // extremum of the raw scores over the allowed keys (max for c >= 0, min for
+                // c < 0); disallowed keys of a partial chunk take the fill value first
+                auto extremum = [&](auto op3, auto op2) -> float {
+                    if (!masked) {
+                        float e[8];  // eight chains of three-input max/min
 #pragma unroll
-                    for (int i = 0; i < 128; ++i) s[i] = (i < lim) ? s[i] : fill;
-                }
-                // extremum of the raw scores over the allowed keys (max for c >= 0, min
-                // for c < 0), times c: eight chains of three-input max/min
-                float e[8];
-                if (c >= 0.f) {
+                        for (int k = 0; k < 8; ++k) {
+                            e[k] = op3(s[k], s[k + 8], s[k + 16]);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        e[k] = max3(s[k], s[k + 8], s[k + 16]);
-#pragma unroll
-                        for (int i = 3; i < 15; i += 2) e[k] = max3(e[k], s[k + 8 * i], s[k + 8 * i + 8]);
-                        e[k] = fmaxf(e[k], s[k + 120]);
+                            for (int i = 3; i < 15; i += 2) e[k] = op3(e[k], s[k + 8 * i], s[k + 8 * i + 8]);
+                            e[k] = op2(e[k], s[k + 120]);
+                        }
+                        return op2(op3(e[0], e[1], e[2]), op3(e[3], e[4], op3(e[5], e[6], e[7])));
                     }
-                    e[0] = fmaxf(max3(e[0], e[1], e[2]), max3(e[3], e[4], max3(e[5], e[6], e[7])));
-                } else {
+                    float acc = fill;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        e[k] = min3(s[k], s[k + 8], s[k + 16]);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (chunk_empty(ch)) continue;
+                        const int b0 = ch * 32;
+                        if (!chunk_full(ch)) {
 #pragma unroll
-                        for (int i = 3; i < 15; i += 2) e[k] = min3(e[k], s[k + 8 * i], s[k + 8 * i + 8]);
-                        e[k] = fminf(e[k], s[k + 120]);
+                            for (int i = 0; i < 32; ++i) s[b0 + i] = (b0 + i < lim) ? s[b0 + i] : fill;
+                        }
+                        float e[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            e[k] = op3(s[b0 + k], s[b0 + k + 4], s[b0 + k + 8]);
+                            e[k] = op3(e[k], s[b0 + k + 12], s[b0 + k + 16]);
+                            e[k] = op3(e[k], s[b0 + k + 20], s[b0 + k + 24]);
+                            e[k] = op2(e[k], s[b0 + k + 28]);
+                        }
+                        acc = op3(acc, op3(e[0], e[1], e[2]), e[3]);
                     }
-                    e[0] = fminf(min3(e[0], e[1], e[2]), min3(e[3], e[4], min3(e[5], e[6], e[7])));
-                }
+                    return acc;
+                };
+                float e[1];
+                if (c >= 0.f)
+                    e[0] = extremum([](float x, float y, float z) { return max3(x, y, z); },
+                                    [](float x, float y) { return fmaxf(x, y); });
+                else
+                    e[0] = extremum([](float x, float y, float z) { return min3(x, y, z); },
+                                    [](float x, float y) { return fminf(x, y); });
                 const float mx = (lim <= 0) ? kNegInf : (c == 0.f ? 0.f : e[0] * c);
                 // Deferred rescaling: move the reference max only when the block's max
                 // exceeds it by more than 8 (a factor 256), which keeps every p <= 256.
@@ -680,27 +735,52 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 // disallowed key gets the exponent -inf, i.e. p = 0, for any sign of c.
                 const float neg_m = (m == kNegInf) ? 0.f : -m;
                 float ls0 = 0.f, ls1 = 0.f;
-                auto exp_range = [&](int ch0, int ch1) {
+                // the pairs of a chunk that take the polynomial, spread over the chunk
+                auto use_poly = [](int ch, int i) { return ((i * 5 + ch * 3) & 15) < C::kPolyPairs; };
+                // one 32-key chunk: P = 2^(c s - m) as bf16 pairs; with kSelect, keys at or
+                // past lim get the exponent -inf (p = 0 for either sign of c)
+                auto exp_chunk = [&](auto select_c, int ch) {
+                    constexpr bool kSelect = decltype(select_c)::value;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int j = ch * 32 + 2 * i;
+                        float x0, x1, p0, p1;
+                        fma2(s[j], s[j + 1], c, c, neg_m, neg_m, x0, x1);
+                        if constexpr (kSelect) {
+                            x0 = (j < lim) ? x0 : kNegInf;
+                            x1 = (j + 1 < lim) ? x1 : kNegInf;
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        } else if (use_poly(ch, i)) {
+                            exp2_poly2(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        add2(ls0, ls1, p0, p1, ls0, ls1);
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st16(s_addr + ch * 16, pk);
+                };
+                auto exp_range = [&](auto masked_c, int ch0, int ch1) {
+                    constexpr bool kMasked = decltype(masked_c)::value;
 #pragma unroll
                     for (int ch = ch0; ch < ch1; ++ch) {
-                        uint32_t pk[16];
+                        if (!kMasked || chunk_full(ch)) {
+                            exp_chunk(std::false_type{}, ch);
+                        } else if (chunk_empty(ch)) {
+                            uint32_t pk[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int j = ch * 32 + 2 * i;
-                            float x0, x1;
-                            fma2(s[j], s[j + 1], c, c, neg_m, neg_m, x0, x1);
-                            if (masked) {
-                                x0 = (j < lim) ? x0 : kNegInf;
-                                x1 = (j + 1 < lim) ? x1 : kNegInf;
-                            }
-                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                            add2(ls0, ls1, p0, p1, ls0, ls1);
-                            pk[i] = pack_bf16x2(p0, p1);
+                            for (int i = 0; i < 16; ++i) pk[i] = 0u;  // two bf16 zeros
+                            tmem_st16(s_addr + ch * 16, pk);
+                        } else {
+                            exp_chunk(std::true_type{}, ch);
                         }
-                        tmem_st16(s_addr + ch * 16, pk);
                     }
                 };
-                exp_range(0, 2);
+                if (masked) exp_range(std::true_type{}, 0, 2);
+                else exp_range(std::false_type{}, 0, 2);
                 // O rescale: PV of the previous block is complete, because this block's S
                 // was issued after it.
                 if (it > 0 && __any_sync(0xffffffffu, grow)) {
@@ -716,7 +796,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                     }
                 }
                 // second half: keys 64..127
-                exp_range(2, 4);
+                if (masked) exp_range(std::true_type{}, 2, 4);
+                else exp_range(std::false_type{}, 2, 4);
                 l += ls0 + ls1;
                 tmem_wait_st();
                 tc_fence_before();
