@@ -26,6 +26,7 @@
 
 #include "fwd_params.h"
 #include "launch.h"
+#include "exp2_poly.cuh"
 #include "ptx_sm100.cuh"
 
 #ifndef GQA_EXP_POLY_PAIRS
@@ -84,31 +85,6 @@ struct FwdCfg {
     __host__ __device__ static constexpr int s_col(int t) { return t * 128; }
     __host__ __device__ static constexpr int o_col(int t) { return NT * 128 + t * HD; }
 };
-
-// 2^x on the FMA and integer pipes, for a share of the exponentials so that they do not
-// all queue on the special-function unit.  Cody-Waite reduction x = j + f with j = rint(x)
-// (the 1.5 * 2^23 rounding constant puts j in the low mantissa bits of t), then
-// 2^f ~ 1 + f (c1 + f (c2 + f c3)) on [-1/2, 1/2]: a degree-3 fit minimising the relative
-// error with the constant term held at 1, max relative error 1.02e-4 (the bf16 rounding
-// of P is 2^-9 = 1.95e-3); 2^j is added to the exponent field.  x is clamped at -126 so the
-// exponent cannot underflow (the result there is 2^-126 instead of a smaller number);
-// inputs are at most 8 (the deferred-rescale bound), far below overflow.  Only for finite x:
-// masked keys keep the exact zero of the special-function path.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-    constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-    constexpr float c1 = 0.6932829022407532f, c2 = 0.24221095442771912f, c3 = 0.055008936673402786f;
-    x0 = fmaxf(x0, -126.f);
-    x1 = fmaxf(x1, -126.f);
-    float t0, t1, r0, r1, f0, f1, q0, q1;
-    add2(x0, x1, kRound, kRound, t0, t1);
-    add2(t0, t1, -kRound, -kRound, r0, r1);
-    add2(x0, x1, -r0, -r1, f0, f1);
-    fma2(f0, f1, c3, c3, c2, c2, q0, q1);
-    fma2(q0, q1, f0, f1, c1, c1, q0, q1);
-    fma2(q0, q1, f0, f1, 1.f, 1.f, q0, q1);
-    y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
 
 template <uint32_t R>
 __device__ __forceinline__ void regs_inc() {
