@@ -84,9 +84,9 @@ def kernel_hash():
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_for(workload_key):
+def traffic_for(workload_key, pack_gqa, num_splits):
     """DRAM bytes per launch from a committed ncu capture, if it was taken on the current
-    kernel source; else None."""
+    kernel source with the same resolved pack / split choice; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
@@ -94,7 +94,9 @@ def traffic_for(workload_key):
     if t.get("kernel_sha256_16") != kernel_hash():
         return None
     e = t.get("workloads", {}).get(workload_key)
-    return None if e is None else e.get("dram_bytes_per_launch")
+    if e is None or e.get("pack_gqa") != pack_gqa or e.get("num_splits") != num_splits:
+        return None
+    return e.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
@@ -346,7 +348,7 @@ def run_gpu(args, cfg):
         unit = "TFLOP/s"
         e2e_value = world * fl / (e2e_ms / 1e3) / 1e12
     roof["peak_source"] = f"{peak_src}:" + ("hbm_gbs" if decode_like else pk_key)
-    roof["traffic"] = traffic_for(cfg["name"])
+    roof["traffic"] = traffic_for(cfg["name"], pack, splits)
     roof["kernel"] = "gqa_fwd_kernel"
 
     tokens = B * (Sq if Sq > 1 else 1)

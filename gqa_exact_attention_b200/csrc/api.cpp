@@ -54,12 +54,17 @@ void padded_rows(int Sq, int g, long long* unpacked, long long* packed) {
     *packed = P >= 1 ? (long long)ceil_div(Sq, P) * kBlockM : (1ll << 62);
 }
 
-int choose_pack(int Sq, int Hq, int Hk) {
+// Pack when it pads fewer tile rows.  Causal attention also packs at equal rows: a unit's
+// two packed tiles cover adjacent short position ranges whose diagonals fall in the same
+// key block, so both tiles finish on the same block, while two 128-position tiles end a
+// block apart and the unit's last block runs one tile alone (measured on B200, causal:
+// +6 % at B=64 S=2048, +16 % at S=1024, +15 % at d=64, within 1.5 % at S=16384).
+int choose_pack(int Sq, int Hq, int Hk, int causal) {
     const int g = Hq / Hk;
     if (g == 1 || g > kBlockM) return 0;
     long long un, pk;
     padded_rows(Sq, g, &un, &pk);
-    return pk < un ? 1 : 0;
+    return (pk < un || (causal && pk == un)) ? 1 : 0;
 }
 
 // Fill everything except the split count from the shape and the pack choice.
@@ -110,8 +115,7 @@ int clamp_splits(int s, int kv_blocks) {
 
 Plan resolve(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal, int pack, int splits,
              int num_sms) {
-    (void)causal;
-    if (pack < 0) pack = choose_pack(Sq, Hq, Hk);
+    if (pack < 0) pack = choose_pack(Sq, Hq, Hk, causal);
     Plan pl = make_plan(B, Sq, Sk, Hq, Hk, pack);
     pl.splits = clamp_splits(splits <= 0 ? choose_splits(pl, d, num_sms) : splits, pl.kv_blocks);
     pl.units *= pl.splits;

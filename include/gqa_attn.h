@@ -105,8 +105,9 @@ GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, flo
  * H100 ("解锁Stable Diffusion效率瓶颈…", "动态批量调度" and "三步优化检查清单";
  * "优化GQA在Flash-Attention中的批量敏感性", strategy 2 and "参数组合"; "為什么 GQA 推理吞吐
  * 先升后降…", "修復" table); this rule is re-derived for B200 instead: pack when it
- * computes fewer padded tile rows, split the key axis when the (batch, head, q-tile)
- * units alone cannot fill the SMs.
+ * computes fewer padded tile rows (causal: also at equal rows, since the two packed tiles
+ * of a unit then end on the same key block), split the key axis when the (batch, head,
+ * q-tile) units alone cannot fill the SMs.
  */
 GQA_API gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
                            int num_sms, int* pack_gqa, int* num_splits);

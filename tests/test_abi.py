@@ -89,8 +89,12 @@ def test_heuristic_pack():
     assert G.gqa_attn_choose(32, 1, 2048, 32, 8, 128, 0)[0] == 1
     # ragged short query (77 positions): packing pads fewer rows
     assert G.gqa_attn_choose(4, 77, 4096, 32, 8, 128, 0)[0] == 1
-    # long prefill, tile-aligned: no packing (equal rows, less causal waste)
-    assert G.gqa_attn_choose(64, 2048, 2048, 32, 8, 128, 1)[0] == 0
+    # long prefill, tile-aligned (equal padded rows): causal packs (the two tiles of a
+    # unit end on the same key block), non-causal does not
+    assert G.gqa_attn_choose(64, 2048, 2048, 32, 8, 128, 1)[0] == 1
+    assert G.gqa_attn_choose(64, 2048, 2048, 32, 8, 128, 0)[0] == 0
+    # packing would pad more rows (g = 3: 42 positions per tile): no packing, causal or not
+    assert G.gqa_attn_choose(2, 2048, 2048, 6, 2, 128, 1)[0] == 0
     # MHA never packs
     assert G.gqa_attn_choose(4, 77, 4096, 32, 32, 128, 0)[0] == 0
 
