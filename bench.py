@@ -9,8 +9,9 @@ One step = one forward over the whole batch.  Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the only reference this project has) on the
 box's host cores, on bounded samples of the same workload.  Other flags (--B, --Sq, ...)
-select another shape for ad-hoc measurement; ``--sweep prefill|decode`` prints one line
-per configuration of the batch-sensitivity sweep or the decode grid.
+select another shape for ad-hoc measurement; ``--sweep prefill|decode|kvcache`` prints one line
+per configuration of the batch-sensitivity sweep, the decode grid, or the KV-cache entry
+point (per-sequence lengths, bf16 output).
 """
 from __future__ import annotations
 
@@ -433,6 +434,8 @@ def run_sweep(args):
     G.load()
     stream = torch.cuda.current_stream()
     peaks, _ = load_peaks()
+    if args.sweep == "kvcache":
+        return run_sweep_kvcache(args, peaks)
     if args.sweep == "prefill":
         cases = [(B, 2048, 2048, c, pk, sp) for B in (16, 32, 64, 128, 256) for c in (1, 0)
                  for (pk, sp) in [(-1, 0), (0, 1), (1, 1), (0, 2), (1, 2), (0, 4), (1, 4)]]
@@ -480,6 +483,60 @@ def run_sweep(args):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep_kvcache(args, peaks):
+    """Kernel-only timings of gqa_attn_fwd_kvcache: decode against a KV cache of capacity
+    8192 whose sequences have seeded lengths uniform in [1, 8192] (B 32/128/256), fp32 and
+    bf16 output; and the prefill shape (B=16, S=2048) with bf16 output.  Bytes and flops
+    count each sequence's own keys."""
+    import numpy as np
+    import torch
+
+    import gqa_exact_attention_b200 as G
+    import inputs
+    stream = torch.cuda.current_stream()
+    Hq, Hk, d = 32, 8, 128
+    cases = [(B, 1, 8192, 0, "uniform", dt) for B in (32, 128, 256) for dt in ("fp32", "bf16")]
+    cases += [(16, 2048, 2048, c, "full", "bf16") for c in (0, 1)]
+    for (B, Sq, Sk, causal, mix, dt) in cases:
+        q = inputs.device_tensor(1001, inputs.TID_Q, (B, Sq, Hq, d))
+        k = inputs.device_tensor(1001, inputs.TID_K, (B, Sk, Hk, d))
+        v = inputs.device_tensor(1001, inputs.TID_V, (B, Sk, Hk, d))
+        rng = np.random.default_rng(7000 + B)
+        lens = rng.integers(1, Sk + 1, size=B) if mix == "uniform" else np.full(B, Sk)
+        sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        odt = torch.bfloat16 if dt == "bf16" else torch.float32
+        out = torch.empty((B, Sq, Hq, d), dtype=odt, device="cuda")
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
+
+        def step():
+            G.gqa_attn_fwd_kvcache(q, k, v, sl, out=out, lse=lse, causal=causal, stream=stream)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if G.gqa_attn_device_status(reset=True) != 0:
+            raise SystemExit("an in-kernel bounded wait timed out")
+        ms = e0.elapsed_time(e1) / args.steps
+        keys = int(lens.sum())
+        osz = 2 if dt == "bf16" else 4
+        by = 2 * B * Sq * Hq * d + 2 * 2 * keys * Hk * d + osz * B * Sq * Hq * d + 4 * B * Hq * Sq
+        fl = sum(flops(1, Sq, int(L), Hq, d, causal) for L in lens)
+        line = {"sweep": "kvcache", "B": B, "Sq": Sq, "Sk_capacity": Sk, "lengths": mix,
+                "mean_length": round(float(lens.mean()), 1), "causal": bool(causal), "out": dt,
+                "ms": round(ms, 4), "hbm_gbs": round(by / ms / 1e6, 1),
+                "frac_of_measured_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 3),
+                "tflops": round(fl / ms / 1e9, 1),
+                "frac_of_measured_bf16": round(fl / ms / 1e9 / peaks["bf16_tflops"], 3)}
+        print(json.dumps(line), flush=True)
+        del q, k, v, out, lse
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -497,7 +554,7 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--sweep", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache"], default=None,
                     help="print one line per configuration of the batch sweep or decode grid")
     args = ap.parse_args()
     if args.warmup < 3:

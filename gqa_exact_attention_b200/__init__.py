@@ -72,6 +72,8 @@ def load():
     L.gqa_attn_device_status.restype = i
     L.gqa_attn_fwd_noalloc.argtypes = [p, p, p, p, p, i, i, i, i, i, i, f, i, i, i, p]
     L.gqa_attn_fwd_noalloc.restype = i
+    L.gqa_attn_fwd_kvcache.argtypes = [p, p, p, p, p, i, p, i, i, i, i, i, i, f, i, i, i, p]
+    L.gqa_attn_fwd_kvcache.restype = i
     _lib = L
     return L
 
@@ -158,3 +160,55 @@ def gqa_attn_fwd_noalloc(q, k, v, out, lse, scale=None, causal=False, pack_gqa=-
     return gqa_attn_fwd(q, k, v, out=out, lse=lse, scale=scale, causal=causal,
                         pack_gqa=pack_gqa, num_splits=num_splits, stream=stream,
                         _entry="gqa_attn_fwd_noalloc")
+
+
+GQA_OUT_F32 = 0
+GQA_OUT_BF16 = 1
+
+
+def gqa_attn_fwd_kvcache(q, k_cache, v_cache, cache_seqlens=None, out=None, lse=None,
+                         out_dtype=None, scale=None, causal=False, pack_gqa=-1, num_splits=0,
+                         stream=None):
+    """out, lse = gqa_attn_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, ...).
+
+    k_cache, v_cache: bf16 [B, Sk, Hk, d] (Sk = the cache's capacity per sequence);
+    cache_seqlens: int32 CUDA tensor [B] (sequence b uses keys [0, cache_seqlens[b]),
+    clamped to [0, Sk]) or None for full length.  out is fp32 or bf16 [B, Sq, Hq, d]
+    (``out_dtype`` torch.float32 / torch.bfloat16 when out is not given; default fp32).
+    Causal masks are bottom-right aligned to each sequence's own length.
+    """
+    import torch
+
+    B, Sq, Hq, d = q.shape
+    Sk, Hk = k_cache.shape[1], k_cache.shape[2]
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if k_cache.shape != v_cache.shape or k_cache.shape[0] != B or k_cache.shape[3] != d:
+        raise ValueError("k_cache and v_cache must be [B, Sk, Hk, d] matching q")
+    if cache_seqlens is not None:
+        if (cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_contiguous()
+                or cache_seqlens.device != q.device or tuple(cache_seqlens.shape) != (B,)):
+            raise ValueError("cache_seqlens must be a contiguous int32 tensor [B] on q's device")
+    if out is None:
+        dt = torch.float32 if out_dtype is None else out_dtype
+        out = torch.empty((B, Sq, Hq, d), dtype=dt, device=q.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or not out.is_contiguous() \
+            or out.device != q.device or tuple(out.shape) != (B, Sq, Hq, d):
+        raise ValueError("out must be a contiguous fp32 or bf16 tensor [B, Sq, Hq, d] on q's device")
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("lse must be a contiguous fp32 tensor [B, Hq, Sq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    code = GQA_OUT_BF16 if out.dtype == torch.bfloat16 else GQA_OUT_F32
+    with torch.cuda.device(q.device):
+        _check(load().gqa_attn_fwd_kvcache(
+            q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+            None if cache_seqlens is None else cache_seqlens.data_ptr(), out.data_ptr(), code,
+            lse.data_ptr(), B, Sq, Sk, Hq, Hk, d, float(scale), int(bool(causal)),
+            int(pack_gqa), int(num_splits), stream.cuda_stream))
+    return out, lse

@@ -161,17 +161,21 @@ bool encode_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, in
 
 // fp32 output [Bs, S, H, d] (Bs = B, or splits * B for the partials) as a 4-D map
 // (d, H, S, Bs) for TMA stores: 128-byte swizzle, box (32, box_h, box_s, 1).
+// Output map for the epilogue's TMA stores: fp32 with 32-column boxes, or bf16 with
+// 64-column boxes; either way a box row is 128 bytes (the 128-byte swizzle span).
 bool encode_out(CUtensorMap* m, const void* ptr, int Bs, int S, int H, int d, int box_h,
-                int box_s) {
+                int box_s, bool bf16 = false) {
     EncodeTiled enc = get_encode_tiled();
     if (!enc) return false;
+    const cuuint64_t es = bf16 ? 2 : 4;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)Bs};
-    cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)S * H * d * 4};
-    cuuint32_t box[4] = {32, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
+    cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)S * H * d * es};
+    cuuint32_t box[4] = {bf16 ? 64u : 32u, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 struct DeviceInfo {
@@ -256,6 +260,103 @@ long long timeout_ns() {
     return ms * 1000000ll;
 }
 
+// The forward behind gqa_attn_fwd and gqa_attn_fwd_kvcache.  out is fp32 or, with
+// out_bf16, bf16; seqlens_k (device, nullable) gives each sequence's key count.
+gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seqlens_k, void* out,
+                    bool out_bf16, float* lse, int B, int Sq, int Sk, int Hq, int Hk, int d,
+                    float scale, int causal, int pack_gqa, int num_splits, void* stream_ptr) {
+    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
+    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
+    if (st != GQA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+        return GQA_ERR_ALIGN;
+    if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) != 0) return GQA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return GQA_ERR_SHAPE;
+    int dev = 0;
+    DeviceInfo info;
+    st = device_info(&dev, &info);
+    if (st != GQA_OK) return st;
+    if (!info.ok) return GQA_ERR_ARCH;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+
+    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms);
+    const int g = Hq / Hk;
+
+    gqa::FwdParams p{};
+    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM) ||
+        !encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
+        !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
+        return GQA_ERR_CUDA;
+    p.out = out_bf16 ? nullptr : static_cast<float*>(out);
+    p.out_bf16 = out_bf16 ? static_cast<uint16_t*>(out) : nullptr;
+    p.seqlens_k = seqlens_k;
+    p.lse = lse;
+    p.B = B;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.Hq = Hq;
+    p.Hk = Hk;
+    p.g = g;
+    p.pack = pl.pack;
+    p.pos_per_tile = pl.pos_per_tile;
+    p.rows_valid = pl.rows_valid;
+    p.causal = causal ? 1 : 0;
+    p.num_splits = pl.splits;
+    p.n_hg = pl.n_hg;
+    p.n_mt = pl.n_mt;
+    p.n_units = (int)pl.units;
+    p.batch_window = batch_window(B, Sk, Hk, d);
+    set_unit_divisors(&p, B);
+    p.kv_blocks = pl.kv_blocks;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.div_g = gqa::make_fastdiv((uint32_t)g);
+    p.status = nullptr;
+    p.timeout_ns = timeout_ns();
+
+    void* ws = nullptr;
+    if (pl.splits > 1) {
+        const size_t rows = (size_t)B * Hq * Sq;
+        const size_t bytes = (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
+        if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
+        cudaMemPool_t pool = workspace_pool(dev);
+        if (pool == nullptr || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GQA_ERR_ALLOC;
+        }
+        p.o_part = static_cast<float*>(ws);
+        p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
+    }
+    if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
+                    pl.splits > 1 ? pl.splits * B : B, Sq, Hq, d, pl.pack ? g : 1,
+                    pl.pack ? pl.pos_per_tile : kBlockM, pl.splits == 1 && out_bf16)) {
+        if (ws) cudaFreeAsync(ws, stream);
+        return GQA_ERR_CUDA;
+    }
+
+    const int slots = info.sms * gqa::fwd_ctas_per_sm(d, pl.nt);
+    const int grid = (int)(pl.units < slots ? pl.units : slots);
+    if (gqa::launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) {
+        if (ws) cudaFreeAsync(ws, stream);
+        return GQA_ERR_CUDA;
+    }
+    if (pl.splits > 1) {
+        gqa::CombineParams c{};
+        c.o_part = p.o_part;
+        c.lse_part = p.lse_part;
+        c.out = p.out;
+        c.out_bf16 = p.out_bf16;
+        c.lse = lse;
+        c.B = B;
+        c.Sq = Sq;
+        c.Hq = Hq;
+        c.num_splits = pl.splits;
+        cudaError_t e = gqa::launch_combine(c, d, info.sms, stream);
+        cudaFreeAsync(ws, stream);
+        if (e != cudaSuccess) return GQA_ERR_CUDA;
+    }
+    return GQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -299,93 +400,18 @@ size_t gqa_attn_workspace_bytes(int B, int Sq, int Sk, int Hq, int Hk, int d, in
 
 gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out, float* lse,
                         int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
-                        int pack_gqa, int num_splits, void* stream_ptr) {
-    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
-    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
-    if (st != GQA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
-        return GQA_ERR_ALIGN;
-    if (!std::isfinite(scale)) return GQA_ERR_SHAPE;
-    int dev = 0;
-    DeviceInfo info;
-    st = device_info(&dev, &info);
-    if (st != GQA_OK) return st;
-    if (!info.ok) return GQA_ERR_ARCH;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+                        int pack_gqa, int num_splits, void* stream) {
+    return fwd_impl(q, k, v, nullptr, out, false, lse, B, Sq, Sk, Hq, Hk, d, scale, causal,
+                    pack_gqa, num_splits, stream);
+}
 
-    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms);
-    const int g = Hq / Hk;
-
-    gqa::FwdParams p{};
-    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM) ||
-        !encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
-        !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
-        return GQA_ERR_CUDA;
-    p.out = out;
-    p.lse = lse;
-    p.B = B;
-    p.Sq = Sq;
-    p.Sk = Sk;
-    p.Hq = Hq;
-    p.Hk = Hk;
-    p.g = g;
-    p.pack = pl.pack;
-    p.pos_per_tile = pl.pos_per_tile;
-    p.rows_valid = pl.rows_valid;
-    p.causal = causal ? 1 : 0;
-    p.num_splits = pl.splits;
-    p.n_hg = pl.n_hg;
-    p.n_mt = pl.n_mt;
-    p.n_units = (int)pl.units;
-    p.batch_window = batch_window(B, Sk, Hk, d);
-    set_unit_divisors(&p, B);
-    p.kv_blocks = pl.kv_blocks;
-    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    p.div_g = gqa::make_fastdiv((uint32_t)g);
-    p.status = nullptr;
-    p.timeout_ns = timeout_ns();
-
-    void* ws = nullptr;
-    if (pl.splits > 1) {
-        const size_t rows = (size_t)B * Hq * Sq;
-        const size_t bytes = (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
-        if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
-        cudaMemPool_t pool = workspace_pool(dev);
-        if (pool == nullptr || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess) {
-            cudaGetLastError();
-            return GQA_ERR_ALLOC;
-        }
-        p.o_part = static_cast<float*>(ws);
-        p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
-    }
-    if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
-                    pl.splits > 1 ? pl.splits * B : B, Sq, Hq, d, pl.pack ? g : 1,
-                    pl.pack ? pl.pos_per_tile : kBlockM)) {
-        if (ws) cudaFreeAsync(ws, stream);
-        return GQA_ERR_CUDA;
-    }
-
-    const int slots = info.sms * gqa::fwd_ctas_per_sm(d, pl.nt);
-    const int grid = (int)(pl.units < slots ? pl.units : slots);
-    if (gqa::launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) {
-        if (ws) cudaFreeAsync(ws, stream);
-        return GQA_ERR_CUDA;
-    }
-    if (pl.splits > 1) {
-        gqa::CombineParams c{};
-        c.o_part = p.o_part;
-        c.lse_part = p.lse_part;
-        c.out = out;
-        c.lse = lse;
-        c.B = B;
-        c.Sq = Sq;
-        c.Hq = Hq;
-        c.num_splits = pl.splits;
-        cudaError_t e = gqa::launch_combine(c, d, info.sms, stream);
-        cudaFreeAsync(ws, stream);
-        if (e != cudaSuccess) return GQA_ERR_CUDA;
-    }
-    return GQA_OK;
+gqa_status gqa_attn_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                                const int* cache_seqlens, void* out, int out_dtype, float* lse,
+                                int B, int Sq, int Sk, int Hq, int Hk, int d, float scale,
+                                int causal, int pack_gqa, int num_splits, void* stream) {
+    if (out_dtype != GQA_OUT_F32 && out_dtype != GQA_OUT_BF16) return GQA_ERR_SHAPE;
+    return fwd_impl(q, k_cache, v_cache, cache_seqlens, out, out_dtype == GQA_OUT_BF16, lse, B,
+                    Sq, Sk, Hq, Hk, d, scale, causal, pack_gqa, num_splits, stream);
 }
 
 gqa_status gqa_attn_device_status(int reset) {

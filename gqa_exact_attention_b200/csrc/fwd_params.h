@@ -45,12 +45,19 @@ struct FwdParams {
     FastDiv div_window, div_splits, div_hg, div_bw, div_bw_last;
     unsigned int* status;  // status word for bounded-wait timeouts (NULL: the library's own)
     long long timeout_ns;  // limit of each in-kernel wait
+    // KV cache with per-sequence lengths: keys [0, seqlens_k[b]) of batch b are valid
+    // (clamped to [0, Sk]); NULL: every sequence has Sk keys
+    const int* seqlens_k;
+    // bf16 output [B, Sq, Hq, d] instead of out (num_splits == 1; with splits the combine
+    // writes it); NULL: fp32 out.  tm_o then maps it as bf16 with 64-column boxes.
+    uint16_t* out_bf16;
 };
 
 struct CombineParams {
     const float* o_part;
     const float* lse_part;
     float* out;
+    uint16_t* out_bf16;  // non-NULL: write the output as bf16 here instead of out
     float* lse;
     int B, Sq, Hq, num_splits;
 };

@@ -99,6 +99,7 @@ __device__ __forceinline__ void regs_dec() {
 template <int NT>
 struct UnitGeom {
     int b, hg, split, kvh;
+    int sk;         // keys of this batch element (its KV-cache length, else Sk)
     int pos0[NT];   // first query position of tile t
     int n[NT];      // key blocks tile t processes in this split
     int kb_lo;      // first key block of the split
@@ -126,6 +127,7 @@ __device__ __forceinline__ UnitGeom<NT> unit_geom(int u, const FwdParams& p) {
     g.b = b0 + (int)rem;
     const int mt = p.n_mt - 1 - (int)q;
     g.kvh = p.pack ? g.hg : (int)fastdiv((uint32_t)g.hg, p.div_g);
+    g.sk = p.seqlens_k ? min(max(__ldg(p.seqlens_k + g.b), 0), p.Sk) : p.Sk;
     int kb_end[NT];
     int kb_union = 0;
 #pragma unroll
@@ -134,8 +136,9 @@ __device__ __forceinline__ UnitGeom<NT> unit_geom(int u, const FwdParams& p) {
         kb_end[t] = 0;
         if (g.pos0[t] < p.Sq) {
             int last = min(g.pos0[t] + p.pos_per_tile, p.Sq) - 1;
-            int key_end = p.Sk;
-            if (p.causal) key_end = max(0, min(p.Sk, last + 1 + (p.Sk - p.Sq)));
+            // causal: bottom-right aligned to this sequence's own key count
+            int key_end = g.sk;
+            if (p.causal) key_end = max(0, min(g.sk, last + 1 + (g.sk - p.Sq)));
             kb_end[t] = (key_end + kBlockN - 1) / kBlockN;
         }
         kb_union = max(kb_union, kb_end[t]);
@@ -192,10 +195,14 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, c
     constexpr float kLn2 = 0.69314718055994530942f;
     const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
     const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
-    float* orow;
+    float* orow = nullptr;
     float* lrow;
+    uint16_t* bf16_row = nullptr;  // bf16 output row (final output only)
     if (p.num_splits == 1) {
-        orow = p.out + (((size_t)b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
+        if (p.out_bf16)
+            bf16_row = p.out_bf16 + (((size_t)b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
+        else
+            orow = p.out + (((size_t)b * p.Sq + rm.pos) * p.Hq + rm.head) * HD;
         lrow = p.lse + ((size_t)b * p.Hq + rm.head) * p.Sq + rm.pos;
     } else {
         const size_t sb = (size_t)split * p.B + b;
@@ -218,7 +225,16 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, c
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = 0u;
         }
-        if (rm.ok) {
+        if (rm.ok && bf16_row != nullptr) {
+            uint4* dst = reinterpret_cast<uint4*>(bf16_row + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l),
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l),
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l),
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l));
+        } else if (rm.ok) {
             float4* dst = reinterpret_cast<float4*>(orow + ch * 32);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -602,7 +618,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 continue;
             }
             // exclusive key bound of this row (causal: j <= pos + Sk - Sq)
-            const int kmax = p.causal ? min(p.Sk, rm.pos + 1 + (p.Sk - p.Sq)) : p.Sk;
+            const int kmax = p.causal ? min(g.sk, rm.pos + 1 + (g.sk - p.Sq)) : g.sk;
             // A warp whose 32 rows are all padding (short query axis, e.g. decode) only
             // keeps the handshake: its P and O rows feed nothing that is stored.
             const bool idle = __all_sync(0xffffffffu, !rm.ok);
@@ -840,6 +856,51 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
                 const int hcoord = p.pack ? g.hg * p.g : g.hg;
                 const int bcoord = p.num_splits == 1 ? g.b : g.split * p.B + g.b;
+                // bf16 output (final output only): a stage row holds 64 bf16 columns, filled
+                // from two 32-column TMEM chunks, then one TMA store of 64 columns
+                const bool bf16_out = p.out_bf16 != nullptr && p.num_splits == 1;
+                if (bf16_out) {
+#pragma unroll
+                    for (int ch = 0; ch < HD / 32; ++ch) {
+                        uint32_t r[32];
+                        if (has && !idle) {
+                            tmem_ld32(o_addr + ch * 32, r);
+                            tmem_wait_ld();
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) r[i] = 0u;
+                        }
+                        if (has && ch == HD / 32 - 1) {
+                            tc_fence_before();
+                            mbar_arrive(o_empty(t));
+                        }
+                        const int half = ch & 1;
+                        if (half == 0) {
+                            if (issuer) bulk_wait_read_all();
+                            named_bar_sync(kEpiBar, 128);
+                        }
+                        const uint32_t dst = sO + row * 128;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t a = dst + ((uint32_t)((half * 4 + j) ^ (row & 7)) << 4);
+                            const float* f = reinterpret_cast<const float*>(r) + 8 * j;
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                                         "r"(pack_bf16x2(f[0] * inv_l, f[1] * inv_l)),
+                                         "r"(pack_bf16x2(f[2] * inv_l, f[3] * inv_l)),
+                                         "r"(pack_bf16x2(f[4] * inv_l, f[5] * inv_l)),
+                                         "r"(pack_bf16x2(f[6] * inv_l, f[7] * inv_l))
+                                         : "memory");
+                        }
+                        if (half == 1) {
+                            fence_proxy_async_smem();
+                            named_bar_sync(kEpiBar, 128);
+                            if (issuer) {
+                                tma_store_4d(&p.tm_o, sO, (ch >> 1) * 64, hcoord, g.pos0[t], bcoord);
+                                bulk_commit_group();
+                            }
+                        }
+                    }
+                } else {
 #pragma unroll
                 for (int ch = 0; ch < HD / 32; ++ch) {
                     uint32_t r[32];
@@ -875,6 +936,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                         tma_store_4d(&p.tm_o, sO, ch * 32, hcoord, g.pos0[t], bcoord);
                         bulk_commit_group();
                     }
+                }
                 }
                 if (rm.ok) {
                     if (p.num_splits == 1)
@@ -945,12 +1007,23 @@ __global__ void __launch_bounds__(256) gqa_combine_kernel(const CombineParams p)
         const long long bh = r / p.Sq;
         const long long h = bh % p.Hq;
         const long long b = bh / p.Hq;
-        float* dst = p.out + ((b * p.Sq + i) * p.Hq + h) * HD + lane * kPer;
-        if constexpr (kPer == 4) {
-            *reinterpret_cast<float4*>(dst) =
-                make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        const long long off = ((b * p.Sq + i) * p.Hq + h) * HD + lane * kPer;
+        if (p.out_bf16 != nullptr) {
+            uint16_t* dst = p.out_bf16 + off;
+            if constexpr (kPer == 4) {
+                *reinterpret_cast<uint2*>(dst) = make_uint2(ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                                                            ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv));
+            } else {
+                *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+            }
         } else {
-            *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+            float* dst = p.out + off;
+            if constexpr (kPer == 4) {
+                *reinterpret_cast<float4*>(dst) =
+                    make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+            } else {
+                *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+            }
         }
         if (lane == 0) p.lse[r] = (wsum > 0.f) ? M + __logf(wsum) : kNegInf;
     }

@@ -117,6 +117,46 @@ GQA_API gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d,
 GQA_API size_t gqa_attn_workspace_bytes(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
                                 int pack_gqa, int num_splits);
 
+/* Element type of the output of gqa_attn_fwd_kvcache. */
+typedef enum { GQA_OUT_F32 = 0, GQA_OUT_BF16 = 1 } gqa_out_dtype;
+
+/*
+ * gqa_attn_fwd_kvcache — the forward of gqa_attn_fwd against a KV cache whose sequences
+ * have their own lengths, with an fp32 or bf16 output.
+ *
+ * The pages run GQA inference against a KV cache that grows with autoregressive
+ * generation ("手把手教你理解Llama2的GQA", section "2.1 KV缓存的内存优化"; "PyTorch 性能分析
+ * 深度指南 (第三部分)", section "深度剖析：内存瓶颈与 KV Cache"), over sequences of different
+ * lengths ("解锁Stable Diffusion效率瓶颈…", section "行业应用场景拓展", scenario one), and
+ * recommend BF16 for attention throughput ("PyTorch 性能分析深度指南", closing advice
+ * "混合精度").
+ *
+ *   k_cache, v_cache  bf16 [B, Sk, Hk, d] as k and v of gqa_attn_fwd; Sk is the cache's
+ *                     capacity per sequence.
+ *   cache_seqlens     device int32 [B] or NULL.  Sequence b uses keys [0, L_b) with
+ *                     L_b = cache_seqlens[b] clamped to [0, Sk]; rows past L_b are never
+ *                     read into the result.  NULL: L_b = Sk for every b (then this call
+ *                     equals gqa_attn_fwd with the chosen output type).  Read by the
+ *                     kernels on the device, in stream order; must stay valid until the
+ *                     call's work on the stream is done.
+ *   causal            bottom-right aligned to each sequence's own length: query i of
+ *                     sequence b sees key j iff j < L_b and j <= i + L_b - Sq.  A row with
+ *                     no key (e.g. L_b = 0) gets O = 0 and LSE = -inf.
+ *   out               [B, Sq, Hq, d], fp32 (out_dtype GQA_OUT_F32) or bf16 rounded to
+ *                     nearest even (GQA_OUT_BF16); 16-byte aligned.
+ *   out_dtype         GQA_OUT_F32 or GQA_OUT_BF16; anything else returns GQA_ERR_SHAPE.
+ *   lse               fp32 [B, Hq, Sq] as in gqa_attn_fwd.
+ *   other arguments   as gqa_attn_fwd.  The heuristic sizes splits for the capacity Sk.
+ *
+ * Errors as gqa_attn_fwd, plus GQA_ERR_ALIGN for a cache_seqlens pointer that is not
+ * 4-byte aligned.  Split-KV partials stay fp32 (allocated as for gqa_attn_fwd).
+ */
+GQA_API gqa_status gqa_attn_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                                        const int* cache_seqlens, void* out, int out_dtype,
+                                        float* lse, int B, int Sq, int Sk, int Hq, int Hk, int d,
+                                        float scale, int causal, int pack_gqa, int num_splits,
+                                        void* stream);
+
 /* Static description of a status code. */
 GQA_API const char* gqa_attn_status_string(gqa_status status);
 

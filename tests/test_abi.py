@@ -21,7 +21,8 @@ def declared_symbols():
 def test_header_declares_the_entry_points():
     assert declared_symbols() == sorted([
         "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes",
-        "gqa_attn_status_string", "gqa_attn_device_status", "gqa_attn_fwd_noalloc"])
+        "gqa_attn_status_string", "gqa_attn_device_status", "gqa_attn_fwd_noalloc",
+        "gqa_attn_fwd_kvcache"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -68,6 +69,25 @@ def test_invalid_arguments_return_before_any_launch(kw, code):
     # the pointers are fake: validation must reject before anything dereferences them
     assert fwd_raw(**kw) == code
     assert G.gqa_attn_status_string(code)
+
+
+def kvcache_raw(q=16, k=16, v=16, seqlens=NULL, out=16, out_dtype=0, lse=16, B=1, Sq=8, Sk=8,
+                Hq=4, Hk=2, d=64, scale=0.125, causal=0, pack=-1, splits=0):
+    L = G.load()
+    return L.gqa_attn_fwd_kvcache(q, k, v, seqlens, out, out_dtype, lse, B, Sq, Sk, Hq, Hk, d,
+                                  scale, causal, pack, splits, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(out_dtype=2), 2), (dict(out_dtype=-1), 2),
+    (dict(q=NULL), 1), (dict(out=NULL), 1), (dict(lse=NULL), 1),
+    (dict(seqlens=18), 5), (dict(out=8), 5),
+    (dict(Hq=6, Hk=4), 3), (dict(d=96), 4), (dict(B=0), 2),
+])
+def test_kvcache_invalid_arguments(kw, code):
+    # fake pointers again: rejected before any launch or dereference (a 4-byte-misaligned
+    # cache_seqlens included)
+    assert kvcache_raw(**kw) == code
 
 
 def test_pages_head_constraint_example():
