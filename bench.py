@@ -486,8 +486,9 @@ def run_sweep(args):
 def run_sweep_kvcache(args, peaks):
     """Kernel-only timings of gqa_attn_fwd_kvcache: decode against a KV cache of capacity
     8192 whose sequences have seeded lengths uniform in [1, 8192] (B 32/128/256), fp32 and
-    bf16 output; and the prefill shape (B=16, S=2048) with bf16 output.  Bytes and flops
-    count each sequence's own keys."""
+    bf16 output with the automatic split count, and fp32 with splits 1/2/4/8; and the
+    prefill shape (B=16, S=2048) with bf16 output.  Bytes and flops count each sequence's
+    own keys."""
     import numpy as np
     import torch
 
@@ -495,9 +496,10 @@ def run_sweep_kvcache(args, peaks):
     import inputs
     stream = torch.cuda.current_stream()
     Hq, Hk, d = 32, 8, 128
-    cases = [(B, 1, 8192, 0, "uniform", dt) for B in (32, 128, 256) for dt in ("fp32", "bf16")]
-    cases += [(16, 2048, 2048, c, "full", "bf16") for c in (0, 1)]
-    for (B, Sq, Sk, causal, mix, dt) in cases:
+    cases = [(B, 1, 8192, 0, "uniform", dt, 0) for B in (32, 128, 256) for dt in ("fp32", "bf16")]
+    cases += [(B, 1, 8192, 0, "uniform", "fp32", sp) for B in (32, 128, 256) for sp in (1, 2, 4, 8)]
+    cases += [(16, 2048, 2048, c, "full", "bf16", 0) for c in (0, 1)]
+    for (B, Sq, Sk, causal, mix, dt, sp) in cases:
         q = inputs.device_tensor(1001, inputs.TID_Q, (B, Sq, Hq, d))
         k = inputs.device_tensor(1001, inputs.TID_K, (B, Sk, Hk, d))
         v = inputs.device_tensor(1001, inputs.TID_V, (B, Sk, Hk, d))
@@ -509,7 +511,8 @@ def run_sweep_kvcache(args, peaks):
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
 
         def step():
-            G.gqa_attn_fwd_kvcache(q, k, v, sl, out=out, lse=lse, causal=causal, stream=stream)
+            G.gqa_attn_fwd_kvcache(q, k, v, sl, out=out, lse=lse, causal=causal, num_splits=sp,
+                                   stream=stream)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
@@ -527,6 +530,7 @@ def run_sweep_kvcache(args, peaks):
         by = 2 * B * Sq * Hq * d + 2 * 2 * keys * Hk * d + osz * B * Sq * Hq * d + 4 * B * Hq * Sq
         fl = sum(flops(1, Sq, int(L), Hq, d, causal) for L in lens)
         line = {"sweep": "kvcache", "B": B, "Sq": Sq, "Sk_capacity": Sk, "lengths": mix,
+                "num_splits": sp if sp > 0 else "auto",
                 "mean_length": round(float(lens.mean()), 1), "causal": bool(causal), "out": dt,
                 "ms": round(ms, 4), "hbm_gbs": round(by / ms / 1e6, 1),
                 "frac_of_measured_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 3),

@@ -107,6 +107,21 @@ int choose_splits(const Plan& pl, int d, int num_sms) {
     return best;
 }
 
+// With per-sequence KV lengths the units' work varies from nothing to the capacity, and
+// the plan cannot see the lengths (they live on the device).  Split until there are at
+// least kVarlenUnitsPerSlot units per CTA slot: a slot then sums several units of
+// unrelated length, and the longest sequence is cut into that many pieces.  Never fewer
+// splits than the dense model picks for the capacity.
+int choose_splits_varlen(const Plan& pl, int d, int num_sms) {
+    constexpr long long kVarlenUnitsPerSlot = 3;  // fitted on B200: uniform lengths, B 32-256
+    const long long slots = (long long)num_sms * gqa::fwd_ctas_per_sm(d, pl.nt);
+    const int smax = pl.kv_blocks < kMaxSplits ? pl.kv_blocks : kMaxSplits;
+    int s = 1;
+    while (s < smax && pl.units * s < kVarlenUnitsPerSlot * slots) ++s;
+    const int dense = choose_splits(pl, d, num_sms);
+    return s > dense ? s : dense;
+}
+
 int clamp_splits(int s, int kv_blocks) {
     if (s > kv_blocks) s = kv_blocks;
     if (s > kMaxSplits) s = kMaxSplits;
@@ -114,10 +129,11 @@ int clamp_splits(int s, int kv_blocks) {
 }
 
 Plan resolve(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal, int pack, int splits,
-             int num_sms) {
+             int num_sms, bool varlen = false) {
     if (pack < 0) pack = choose_pack(Sq, Hq, Hk, causal);
     Plan pl = make_plan(B, Sq, Sk, Hq, Hk, pack);
-    pl.splits = clamp_splits(splits <= 0 ? choose_splits(pl, d, num_sms) : splits, pl.kv_blocks);
+    const int auto_splits = varlen ? choose_splits_varlen(pl, d, num_sms) : choose_splits(pl, d, num_sms);
+    pl.splits = clamp_splits(splits <= 0 ? auto_splits : splits, pl.kv_blocks);
     pl.units *= pl.splits;
     return pl;
 }
@@ -279,7 +295,8 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     if (!info.ok) return GQA_ERR_ARCH;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
 
-    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms);
+    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms,
+                            seqlens_k != nullptr);
     const int g = Hq / Hk;
 
     gqa::FwdParams p{};
