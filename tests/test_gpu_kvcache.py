@@ -79,9 +79,15 @@ def test_no_lengths_equals_fwd(causal):
     shp = (4, 300, 700, 32, 8, 128)
     q, k, v = P.device_inputs(6000 + causal, *shp)
     ref, lref = G.gqa_attn_fwd(q, k, v, causal=causal)
-    for lens in (None, [700] * 4):
-        out, lse = run_kv(q, k, v, lens, causal)
-        assert torch.equal(out, ref) and torch.equal(lse, lref)
+    # no lengths: the same plan as gqa_attn_fwd
+    out, lse = run_kv(q, k, v, None, causal)
+    assert torch.equal(out, ref) and torch.equal(lse, lref)
+    # all lengths = capacity: the same values under the same schedule (with lengths given
+    # the automatic split count follows the ragged-length rule, so pin pack and splits)
+    pk, ns = G.gqa_attn_choose(*shp, causal)
+    ref, lref = G.gqa_attn_fwd(q, k, v, causal=causal, pack_gqa=pk, num_splits=ns)
+    out, lse = run_kv(q, k, v, [700] * 4, causal, pk, ns)
+    assert torch.equal(out, ref) and torch.equal(lse, lref)
 
 
 def test_lengths_are_clamped_to_capacity():
