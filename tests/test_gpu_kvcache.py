@@ -3,8 +3,9 @@
 
 The oracle runs each sequence on its own key count (the cache rows [0, L_b)), so causal
 masks are bottom-right aligned to L_b as the entry point defines.  bf16 output must equal
-the fp32 output of the same call rounded to nearest even, bit for bit; with no lengths (or
-all lengths = capacity) the entry point must equal gqa_attn_fwd bit for bit.
+the fp32 output of the same call rounded to nearest even, bit for bit; with no lengths, or
+with all lengths = capacity under the same pack/split schedule, the entry point must equal
+gqa_attn_fwd bit for bit.
 """
 import numpy as np
 import pytest
