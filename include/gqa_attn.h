@@ -149,7 +149,11 @@ typedef enum { GQA_OUT_F32 = 0, GQA_OUT_BF16 = 1 } gqa_out_dtype;
  *   other arguments   as gqa_attn_fwd.  The heuristic sizes splits for the capacity Sk.
  *
  * Errors as gqa_attn_fwd, plus GQA_ERR_ALIGN for a cache_seqlens pointer that is not
- * 4-byte aligned.  Split-KV partials stay fp32 (allocated as for gqa_attn_fwd).
+ * 4-byte aligned.  Split-KV partials stay fp32 (allocated as for gqa_attn_fwd).  With
+ * cache_seqlens given and num_splits = 0, the split count follows a rule for ragged
+ * lengths (about three units per CTA slot, never fewer splits than the dense rule), so
+ * the partials can exceed what gqa_attn_workspace_bytes reports for the same shape; at
+ * most 16 splits of B * Hq * Sq * (d + 1) fp32 values.
  */
 GQA_API gqa_status gqa_attn_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
                                         const int* cache_seqlens, void* out, int out_dtype,
