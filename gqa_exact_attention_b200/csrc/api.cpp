@@ -7,8 +7,10 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstdlib>
 #include <mutex>
+#include <vector>
 
 #include "fwd_params.h"
 #include "launch.h"
@@ -122,6 +124,61 @@ int choose_splits_varlen(const Plan& pl, int d, int num_sms) {
     return s > dense ? s : dense;
 }
 
+// Tuned schedules, read once per process from the text file named by GQA_TUNE_TABLE (as
+// written by the package's autotune module).  One entry per line:
+//   d causal Hq Hk bucket(B) bucket(Sq) bucket(Sk) pack_gqa num_splits [anything else]
+// with bucket(x) = the smallest e such that 2^e >= x.  '#' starts a comment line; lines
+// that do not parse are skipped; a later line for the same key wins.
+struct TuneEntry {
+    int d, causal, Hq, Hk, bB, bSq, bSk, pack, splits;
+};
+
+int bucket(int x) {
+    int e = 0;
+    while (e < 31 && (1ll << e) < x) ++e;
+    return e;
+}
+
+const std::vector<TuneEntry>& tune_table() {
+    static std::vector<TuneEntry> table;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* path = std::getenv("GQA_TUNE_TABLE");
+        if (path == nullptr || *path == '\0') return;
+        FILE* f = std::fopen(path, "r");
+        if (f == nullptr) return;
+        char line[512];
+        while (std::fgets(line, sizeof line, f) != nullptr) {
+            if (line[0] == '#') continue;
+            TuneEntry e{};
+            if (std::sscanf(line, "%d %d %d %d %d %d %d %d %d", &e.d, &e.causal, &e.Hq, &e.Hk,
+                            &e.bB, &e.bSq, &e.bSk, &e.pack, &e.splits) == 9 &&
+                (e.pack == 0 || e.pack == 1) && e.splits >= 1 && (e.causal == 0 || e.causal == 1))
+                table.push_back(e);
+        }
+        std::fclose(f);
+    });
+    return table;
+}
+
+// The tuned (pack, splits) for this shape's bucket, if the table has one that is valid
+// for the shape (packing needs g <= 128).
+bool tuned_choice(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal, int* pack,
+                  int* splits) {
+    const std::vector<TuneEntry>& t = tune_table();
+    const int bB = bucket(B), bSq = bucket(Sq), bSk = bucket(Sk);
+    for (auto it = t.rbegin(); it != t.rend(); ++it) {
+        if (it->d == d && it->causal == causal && it->Hq == Hq && it->Hk == Hk && it->bB == bB &&
+            it->bSq == bSq && it->bSk == bSk) {
+            if (it->pack == 1 && Hq / Hk > kBlockM) return false;
+            *pack = it->pack;
+            *splits = it->splits;
+            return true;
+        }
+    }
+    return false;
+}
+
 int clamp_splits(int s, int kv_blocks) {
     if (s > kv_blocks) s = kv_blocks;
     if (s > kMaxSplits) s = kMaxSplits;
@@ -130,6 +187,14 @@ int clamp_splits(int s, int kv_blocks) {
 
 Plan resolve(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal, int pack, int splits,
              int num_sms, bool varlen = false) {
+    // a tuned schedule replaces the heuristic for fully automatic calls (dense KV only)
+    if (pack < 0 && splits <= 0 && !varlen) {
+        int tp = 0, ts = 0;
+        if (tuned_choice(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, &tp, &ts)) {
+            pack = tp;
+            splits = ts;
+        }
+    }
     if (pack < 0) pack = choose_pack(Sq, Hq, Hk, causal);
     Plan pl = make_plan(B, Sq, Sk, Hq, Hk, pack);
     const int auto_splits = varlen ? choose_splits_varlen(pl, d, num_sms) : choose_splits(pl, d, num_sms);

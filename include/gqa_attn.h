@@ -108,6 +108,15 @@ GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, flo
  * computes fewer padded tile rows (causal: also at equal rows, since the two packed tiles
  * of a unit then end on the same key block), split the key axis when the (batch, head,
  * q-tile) units alone cannot fill the SMs.
+ *
+ * Tuned schedules replace the rule: if the environment variable GQA_TUNE_TABLE names a
+ * table file (written by the package's autotune module; read once per process, at the
+ * first call that needs it), a shape whose bucket (d, causal, Hq, Hk and the power-of-two
+ * buckets of B, Sq, Sk) has an entry gets that entry's pack_gqa / num_splits, validated
+ * for the shape (packing needs Hq/Hk <= 128; splits are clamped to the key blocks).
+ * The same applies to gqa_attn_fwd called with pack_gqa = -1 and num_splits = 0; not to
+ * gqa_attn_fwd_kvcache with per-sequence lengths.  A missing or unreadable file leaves
+ * the rule in place.
  */
 GQA_API gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
                            int num_sms, int* pack_gqa, int* num_splits);
