@@ -122,3 +122,17 @@ def test_many_units_causal_splits(shp, splits):
     o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(shp[-1]), 1)
     out, lse = run(q, k, v, 1, 0, splits)
     P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"{shp} s{splits}")
+
+
+# --- scales other than 1/sqrt(d): a negative scale (the extremum becomes a row minimum) and
+#     a large one (exponents far below -126, the polynomial's clamp), causal and not
+@pytest.mark.parametrize("scale", [-0.09, 1.5])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("pack,splits", [(0, 1), (1, 2), (-1, 0)])
+def test_other_scales(scale, causal, pack, splits):
+    shp = (2, 300, 300, 8, 2, 128)
+    seed = 3400
+    q, k, v = P.device_inputs(seed, *shp)
+    o_ref, l_ref = P.oracle_full(seed, *shp, scale, causal)
+    out, lse = run(q, k, v, causal, pack, splits, scale=scale)
+    P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"scale {scale} c{causal} p{pack} s{splits}")
