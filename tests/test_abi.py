@@ -148,3 +148,7 @@ def test_no_gpu_is_an_error_not_a_fallback():
         pytest.skip("a GPU is present")
     # valid arguments on a machine without a GPU: a CUDA error, never a CPU result
     assert fwd_raw() in (6, 8)
+    assert kvcache_raw() in (6, 8)
+    assert kvcache_raw(seqlens=32, out_dtype=1) in (6, 8)
+    L = G.load()
+    assert L.gqa_attn_fwd_noalloc(16, 16, 16, 16, 16, 1, 8, 8, 4, 2, 64, 0.125, 0, -1, 0, None) in (6, 8)
