@@ -92,8 +92,9 @@ def _check(status: int):
         raise GqaError(status, gqa_attn_status_string(status))
 
 
-def gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, causal, num_sms=148):
-    """The heuristic's (pack_gqa, num_splits) for this shape (host only)."""
+def gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, causal, num_sms=0):
+    """The heuristic's (pack_gqa, num_splits) for this shape, planned for ``num_sms`` SMs
+    (0: the current device's count, as gqa_attn_fwd plans; 148 without a device)."""
     pk, ns = ctypes.c_int(), ctypes.c_int()
     _check(load().gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, int(bool(causal)), num_sms,
                                   ctypes.byref(pk), ctypes.byref(ns)))

@@ -268,7 +268,10 @@ gqa_status device_info(int* dev_out, DeviceInfo* info) {
     static DeviceInfo cache[64];
     static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();  // leave no error pending for the caller's own checks
+        return GQA_ERR_CUDA;
+    }
     *dev_out = dev;
     std::lock_guard<std::mutex> lk(mu);
     if (dev >= 0 && dev < 64 && cache[dev].sms > 0) {
@@ -278,14 +281,25 @@ gqa_status device_info(int* dev_out, DeviceInfo* info) {
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
         return GQA_ERR_CUDA;
+    }
     DeviceInfo di;
     di.sms = sms;
     di.ok = (major == 10 && minor == 0) ? 1 : 0;
     if (dev >= 0 && dev < 64) cache[dev] = di;
     *info = di;
     return GQA_OK;
+}
+
+// SM count the plan assumes when no device is given: the current device's when there is
+// one (what gqa_attn_fwd will plan with), else a B200's 148.
+int planning_sms() {
+    int dev = 0;
+    DeviceInfo info;
+    if (device_info(&dev, &info) == GQA_OK && info.sms > 0) return info.sms;
+    return kDefaultSms;
 }
 
 // Batches per scheduling window: as many as keep the window's K and V within ~48 MB of
@@ -334,18 +348,44 @@ cudaMemPool_t workspace_pool(int dev) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Limit of each in-kernel wait: GQA_WAIT_TIMEOUT_NS (nanoseconds) if set, else
+// GQA_WAIT_TIMEOUT_MS (milliseconds), else 4 s.  Read at every call.
 long long timeout_ns() {
+    if (const char* e = std::getenv("GQA_WAIT_TIMEOUT_NS")) {
+        const long long ns = std::atoll(e);
+        return ns < 1 ? 1 : ns;
+    }
     const char* e = std::getenv("GQA_WAIT_TIMEOUT_MS");
     long long ms = e ? std::atoll(e) : 4000;
     if (ms < 1) ms = 1;
     return ms * 1000000ll;
 }
 
-// The forward behind gqa_attn_fwd and gqa_attn_fwd_kvcache.  out is fp32 or, with
-// out_bf16, bf16; seqlens_k (device, nullable) gives each sequence's key count.
+// Limit of the teardown waits after an abort (copies and MMAs already issued must land
+// before shared and tensor memory are released): never below 1 s, whatever the wait
+// limit, since those operations complete in microseconds unless the device is stuck.
+long long drain_ns(long long wait_ns) { return wait_ns > 1000000000ll ? wait_ns : 1000000000ll; }
+
+// Where the split-KV partials live: the library's stream-ordered pool (scratch ==
+// nullptr), or a fixed caller-side buffer of scratch_bytes that is never allocated or
+// freed here (the allocation-free entry point).
+struct Scratch {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+
+size_t partial_bytes(int splits, int B, int Sq, int Hq, int d) {
+    if (splits <= 1) return 0;
+    return (size_t)splits * (size_t)B * Hq * Sq * ((size_t)d + 1) * sizeof(float);
+}
+
+// The forward behind every entry point.  out is fp32 or, with out_bf16, bf16; seqlens_k
+// (device, nullable) gives each sequence's key count; fixed (nullable) replaces the pool
+// allocation of the split partials.
 gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seqlens_k, void* out,
                     bool out_bf16, float* lse, int B, int Sq, int Sk, int Hq, int Hk, int d,
-                    float scale, int causal, int pack_gqa, int num_splits, void* stream_ptr) {
+                    float scale, int causal, int pack_gqa, int num_splits, void* stream_ptr,
+                    const Scratch* fixed = nullptr) {
     if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
     gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
     if (st != GQA_OK) return st;
@@ -360,8 +400,20 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     if (!info.ok) return GQA_ERR_ARCH;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
 
-    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms,
-                            seqlens_k != nullptr);
+    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms,
+                      seqlens_k != nullptr);
+    if (fixed != nullptr) {
+        // fixed scratch: an automatic split count shrinks until its partials fit (down to
+        // no split, which needs none); an explicit one that does not fit is refused
+        const size_t cap = fixed->ptr ? fixed->bytes : 0;
+        if (num_splits <= 0) {
+            const int s0 = pl.splits;
+            while (pl.splits > 1 && partial_bytes(pl.splits, B, Sq, Hq, d) > cap) --pl.splits;
+            pl.units = pl.units / s0 * pl.splits;
+        } else if (partial_bytes(pl.splits, B, Sq, Hq, d) > cap) {
+            return GQA_ERR_SCRATCH;
+        }
+    }
     const int g = Hq / Hk;
 
     gqa::FwdParams p{};
@@ -394,18 +446,27 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     p.div_g = gqa::make_fastdiv((uint32_t)g);
     p.status = nullptr;
     p.timeout_ns = timeout_ns();
+    p.drain_ns = drain_ns(p.timeout_ns);
 
-    void* ws = nullptr;
+    void* ws = nullptr;  // pool allocation to release after the combine (never with fixed)
     if (pl.splits > 1) {
         const size_t rows = (size_t)B * Hq * Sq;
-        const size_t bytes = (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
-        if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
-        cudaMemPool_t pool = workspace_pool(dev);
-        if (pool == nullptr || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess) {
-            cudaGetLastError();
-            return GQA_ERR_ALLOC;
+        const size_t bytes = partial_bytes(pl.splits, B, Sq, Hq, d);
+        void* part = nullptr;
+        if (fixed != nullptr) {
+            part = fixed->ptr;
+        } else {
+            // host-side fault injection: the allocation fails as it would when the device
+            // is out of memory (nothing is launched)
+            if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
+            cudaMemPool_t pool = workspace_pool(dev);
+            if (pool == nullptr || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess) {
+                cudaGetLastError();
+                return GQA_ERR_ALLOC;
+            }
+            part = ws;
         }
-        p.o_part = static_cast<float*>(ws);
+        p.o_part = static_cast<float*>(part);
         p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
     }
     if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
@@ -433,7 +494,7 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
         c.Hq = Hq;
         c.num_splits = pl.splits;
         cudaError_t e = gqa::launch_combine(c, d, info.sms, stream);
-        cudaFreeAsync(ws, stream);
+        if (ws) cudaFreeAsync(ws, stream);
         if (e != cudaSuccess) return GQA_ERR_CUDA;
     }
     return GQA_OK;
@@ -465,7 +526,7 @@ gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int cau
     if (!pack_gqa || !num_splits) return GQA_ERR_NULL;
     gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, -1, 0);
     if (st != GQA_OK) return st;
-    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal, -1, 0, num_sms > 0 ? num_sms : kDefaultSms);
+    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal, -1, 0, num_sms > 0 ? num_sms : planning_sms());
     *pack_gqa = pl.pack;
     *num_splits = pl.splits;
     return GQA_OK;
@@ -474,10 +535,8 @@ gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int cau
 size_t gqa_attn_workspace_bytes(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
                                 int pack_gqa, int num_splits) {
     if (validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits) != GQA_OK) return 0;
-    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal, pack_gqa, num_splits, kDefaultSms);
-    if (pl.splits <= 1) return 0;
-    const size_t rows = (size_t)B * Hq * Sq;
-    return (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float);
+    Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal, pack_gqa, num_splits, planning_sms());
+    return partial_bytes(pl.splits, B, Sq, Hq, d);
 }
 
 gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, float* out, float* lse,
@@ -513,83 +572,15 @@ gqa_status gqa_attn_device_status(int reset) {
 
 namespace gqa {
 
-// Forward with caller-provided split-KV scratch (no allocation): used by
-// gqa_attn_fwd_noalloc.  Same validation and plan as gqa_attn_fwd.
-gqa_status fwd_with_scratch(const void* q, const void* k, const void* v, float* out, float* lse,
-                            int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
-                            int pack_gqa, int num_splits, void* stream_ptr, void* scratch,
-                            size_t scratch_bytes) {
-    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
-    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
-    if (st != GQA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
-        return GQA_ERR_ALIGN;
-    if (!std::isfinite(scale)) return GQA_ERR_SHAPE;
-    int dev = 0;
-    DeviceInfo info;
-    st = device_info(&dev, &info);
-    if (st != GQA_OK) return st;
-    if (!info.ok) return GQA_ERR_ARCH;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-
-    const Plan pl = resolve(B, Sq, Sk, Hq, Hk, d, causal ? 1 : 0, pack_gqa, num_splits, info.sms);
-    const int g = Hq / Hk;
-    const size_t rows = (size_t)B * Hq * Sq;
-    const size_t need = pl.splits > 1 ? (size_t)pl.splits * rows * ((size_t)d + 1) * sizeof(float) : 0;
-    if (need > 0 && (scratch == nullptr || need > scratch_bytes)) return GQA_ERR_SCRATCH;
-
-    FwdParams p{};
-    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM) ||
-        !encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
-        !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
-        return GQA_ERR_CUDA;
-    p.out = out;
-    p.lse = lse;
-    p.B = B;
-    p.Sq = Sq;
-    p.Sk = Sk;
-    p.Hq = Hq;
-    p.Hk = Hk;
-    p.g = g;
-    p.pack = pl.pack;
-    p.pos_per_tile = pl.pos_per_tile;
-    p.rows_valid = pl.rows_valid;
-    p.causal = causal ? 1 : 0;
-    p.num_splits = pl.splits;
-    p.n_hg = pl.n_hg;
-    p.n_mt = pl.n_mt;
-    p.n_units = (int)pl.units;
-    p.batch_window = batch_window(B, Sk, Hk, d);
-    set_unit_divisors(&p, B);
-    p.kv_blocks = pl.kv_blocks;
-    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    p.div_g = make_fastdiv((uint32_t)g);
-    p.status = nullptr;
-    p.timeout_ns = timeout_ns();
-    if (pl.splits > 1) {
-        p.o_part = static_cast<float*>(scratch);
-        p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
-    }
-    if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
-                    pl.splits > 1 ? pl.splits * B : B, Sq, Hq, d, pl.pack ? g : 1,
-                    pl.pack ? pl.pos_per_tile : kBlockM))
-        return GQA_ERR_CUDA;
-    const int slots = info.sms * fwd_ctas_per_sm(d, pl.nt);
-    const int grid = (int)(pl.units < slots ? pl.units : slots);
-    if (launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) return GQA_ERR_CUDA;
-    if (pl.splits > 1) {
-        CombineParams c{};
-        c.o_part = p.o_part;
-        c.lse_part = p.lse_part;
-        c.out = out;
-        c.lse = lse;
-        c.B = B;
-        c.Sq = Sq;
-        c.Hq = Hq;
-        c.num_splits = pl.splits;
-        if (launch_combine(c, d, info.sms, stream) != cudaSuccess) return GQA_ERR_CUDA;
-    }
-    return GQA_OK;
+gqa_status fwd_fixed_scratch(const void* q, const void* k, const void* v, float* out, float* lse,
+                             int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
+                             int pack_gqa, int num_splits, void* stream, void* scratch,
+                             size_t scratch_bytes) {
+    Scratch fixed;
+    fixed.ptr = scratch;
+    fixed.bytes = scratch_bytes;
+    return fwd_impl(q, k, v, nullptr, out, false, lse, B, Sq, Sk, Hq, Hk, d, scale, causal,
+                    pack_gqa, num_splits, stream, &fixed);
 }
 
 }  // namespace gqa

@@ -45,6 +45,7 @@ struct FwdParams {
     FastDiv div_window, div_splits, div_hg, div_bw, div_bw_last;
     unsigned int* status;  // status word for bounded-wait timeouts (NULL: the library's own)
     long long timeout_ns;  // limit of each in-kernel wait
+    long long drain_ns;    // limit of each teardown wait after an abort (>= 1 s)
     // KV cache with per-sequence lengths: keys [0, seqlens_k[b]) of batch b are valid
     // (clamped to [0, Sk]); NULL: every sequence has Sk keys
     const int* seqlens_k;

@@ -14,10 +14,12 @@ cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, int grid, cudaStream_
 cudaError_t launch_combine(const CombineParams& p, int hd, int num_sms, cudaStream_t stream);
 // Device address of the library's status word on the current device (NULL on error).
 unsigned int* device_status_symbol();
-// The forward with caller-provided split-KV scratch; never allocates (api.cpp).
-gqa_status fwd_with_scratch(const void* q, const void* k, const void* v, float* out, float* lse,
-                            int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
-                            int pack_gqa, int num_splits, void* stream, void* scratch,
-                            size_t scratch_bytes);
+// The forward with its split-KV partials in caller-side fixed scratch of scratch_bytes
+// (never allocates): an automatic split count shrinks to fit, an explicit one that does
+// not fit returns GQA_ERR_SCRATCH (api.cpp).
+gqa_status fwd_fixed_scratch(const void* q, const void* k, const void* v, float* out, float* lse,
+                             int B, int Sq, int Sk, int Hq, int Hk, int d, float scale, int causal,
+                             int pack_gqa, int num_splits, void* stream, void* scratch,
+                             size_t scratch_bytes);
 
 }  // namespace gqa

@@ -20,25 +20,30 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GQA_NOALLOC_SCRATCH_BYTES];
 
 // Host code must not pass g_noalloc_scratch itself (a host-side stand-in, not a device
-// address): its device address is looked up once per device, with that device current.
-struct ScratchAddr {
-    std::once_flag once;
-    void* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
-ScratchAddr g_addr[64];
+// address): its device address is looked up per device, with that device current.  Only
+// a successful look-up is kept, so a call that failed (for instance one made during a
+// stream capture) does not break the device for later calls; they retry.
+constexpr int kMaxDevices = 64;
+std::mutex g_addr_mu;
+void* g_addr[kMaxDevices] = {};
 
 gqa_status scratch_for_current_device(void** out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ERR_CUDA;
-    ScratchAddr& a = g_addr[dev];
-    std::call_once(a.once, [&a] {
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return GQA_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_addr_mu);
+    if (g_addr[dev] == nullptr) {
         void* ptr = nullptr;
-        a.err = cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch);
-        if (a.err == cudaSuccess) a.ptr = ptr;
-    });
-    if (a.err != cudaSuccess || a.ptr == nullptr) return GQA_ERR_CUDA;
-    *out = a.ptr;
+        if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+            cudaGetLastError();  // leave no error pending for the caller's own checks
+            return GQA_ERR_CUDA;
+        }
+        g_addr[dev] = ptr;
+    }
+    *out = g_addr[dev];
     return GQA_OK;
 }
 
@@ -52,7 +57,7 @@ extern "C" gqa_status gqa_attn_fwd_noalloc(const void* q, const void* k, const v
     void* scratch = nullptr;
     gqa_status st = scratch_for_current_device(&scratch);
     if (st != GQA_OK) return st;
-    return gqa::fwd_with_scratch(q, k, v, out, lse, B, Sq, Sk, Hq, Hk, d, scale, causal,
-                                 pack_gqa, num_splits, stream, scratch,
-                                 GQA_NOALLOC_SCRATCH_BYTES);
+    return gqa::fwd_fixed_scratch(q, k, v, out, lse, B, Sq, Sk, Hq, Hk, d, scale, causal,
+                                  pack_gqa, num_splits, stream, scratch,
+                                  GQA_NOALLOC_SCRATCH_BYTES);
 }

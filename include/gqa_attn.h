@@ -99,10 +99,16 @@ GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, flo
                         int pack_gqa, int num_splits, void* stream);
 
 /*
- * The scheduling heuristic alone (host only, no CUDA call): what gqa_attn_fwd uses when
- * pack_gqa = -1 / num_splits = 0.  num_sms is the device's SM count (148 on B200; pass
- * <= 0 for 148).  The pages give four mutually contradictory batch-size tables tuned on
- * H100 ("解锁Stable Diffusion效率瓶颈…", "动态批量调度" and "三步优化检查清单";
+ * The scheduling heuristic alone (no launch, no allocation): what gqa_attn_fwd uses when
+ * pack_gqa = -1 / num_splits = 0.  num_sms is the SM count to plan for (148 on B200);
+ * num_sms <= 0 plans for the current CUDA device's count, as gqa_attn_fwd does, or for
+ * 148 when no device is available (the only CUDA calls made are the device queries).
+ * Compared with the pages' call, which takes tensors and decides inside, this entry point
+ * also takes Hk, causal and num_sms, because the rule depends on the group size, the mask
+ * and the number of SMs to fill.
+ *
+ * The pages give four mutually contradictory batch-size tables tuned on H100
+ * ("解锁Stable Diffusion效率瓶颈…", "动态批量调度" and "三步优化检查清单";
  * "优化GQA在Flash-Attention中的批量敏感性", strategy 2 and "参数组合"; "為什么 GQA 推理吞吐
  * 先升后降…", "修復" table); this rule is re-derived for B200 instead: pack when it
  * computes fewer padded tile rows (causal: also at equal rows, since the two packed tiles
@@ -122,7 +128,12 @@ GQA_API gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d,
                            int num_sms, int* pack_gqa, int* num_splits);
 
 /* Bytes of split-KV scratch gqa_attn_fwd allocates for these arguments (0 when
- * num_splits resolves to 1).  pack_gqa / num_splits follow gqa_attn_fwd's conventions. */
+ * num_splits resolves to 1): num_splits * B * Hq * Sq * (d + 1) * 4 after num_splits is
+ * resolved.  pack_gqa / num_splits follow gqa_attn_fwd's conventions; an automatic split
+ * count is resolved for the current device's SM count (148 without a device), exactly as
+ * gqa_attn_fwd resolves it.  It takes Sk, Hk, causal and pack_gqa besides (B, Sq, Hq, d,
+ * num_splits) because an automatic split count depends on all of them.  Invalid arguments
+ * give 0. */
 GQA_API size_t gqa_attn_workspace_bytes(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
                                 int pack_gqa, int num_splits);
 
@@ -177,6 +188,16 @@ GQA_API const char* gqa_attn_status_string(gqa_status status);
  * Device-side status word of the current device (GQA_OK or GQA_ERR_TIMEOUT), written by
  * kernels whose bounded waits ran out.  Synchronous: it waits for the device.  With
  * reset != 0 the word is cleared after reading.
+ *
+ * Every wait inside the forward kernel (for a copy, an MMA or another warp's hand-off) is
+ * bounded.  The limit is read at each call from the environment: GQA_WAIT_TIMEOUT_NS
+ * (nanoseconds) if set, else GQA_WAIT_TIMEOUT_MS (milliseconds), else 4 s.  A CTA whose
+ * wait runs out sets this word, stops issuing work, lets the copies and MMAs it already
+ * issued complete (waiting at least 1 s for them, whatever the limit), releases its
+ * tensor memory and exits; the rest of the grid notices and exits the same way.  The
+ * call itself has already returned GQA_OK (it is asynchronous), and out / lse are then
+ * partly unwritten: read this word after synchronising when that matters.  Later calls
+ * are unaffected.
  */
 GQA_API gqa_status gqa_attn_device_status(int reset);
 
@@ -196,10 +217,12 @@ GQA_API gqa_status gqa_attn_device_status(int reset);
  *
  * Scratch: the split-KV partials (O_s and lse_s per split) live in one fixed array
  * inside the library, GQA_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads the
- * library, held until the process exits.  A call whose partials need more, i.e.
- * num_splits * B * Hq * Sq * (d + 1) * 4 bytes after num_splits is resolved, returns
- * GQA_ERR_SCRATCH before anything is launched.  With num_splits resolving to 1 no
- * scratch is used.
+ * library, held until the process exits.  The partials need
+ * num_splits * B * Hq * Sq * (d + 1) * 4 bytes.  With num_splits = 0 (automatic) the
+ * chosen split count is lowered until they fit, down to 1, which needs no scratch; so an
+ * automatic call never fails for lack of scratch (it may run with fewer splits than
+ * gqa_attn_fwd would).  An explicit num_splits whose partials do not fit returns
+ * GQA_ERR_SCRATCH before anything is launched.
  *
  * The array is shared by every call on a device and keeps the last call's contents.
  * Nothing in it has to start at zero: every partial element is written before the

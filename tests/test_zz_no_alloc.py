@@ -10,6 +10,7 @@ that both use the scratch, and that a request too large for the scratch is refus
 before anything is launched.  (This file is collected last on purpose.)
 """
 import math
+import os
 
 import numpy as np
 import pytest
@@ -80,3 +81,56 @@ def test_noalloc_refuses_partials_larger_than_the_scratch():
     torch.cuda.synchronize()
     assert (out - ref_out).abs().max().item() <= P.VARIANT_MAX
     assert np.isfinite(lse.cpu().numpy()).all()
+
+
+def test_noalloc_shrinks_an_automatic_split_to_fit_the_scratch():
+    """An automatic split count whose partials would not fit the fixed scratch is lowered
+    (down to no split) instead of failing: a caller that cannot allocate cannot predict
+    the split the library will choose either."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gqa_exact_attention_b200 as G
+    L = G.load()
+    shp = (1, 1024, 65536, 8, 8, 128)
+    B, Sq, Sk, Hq, Hk, d = shp
+    pk, ns = G.gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, 0)
+    assert ns >= 2
+    assert G.gqa_attn_workspace_bytes(B, Sq, Sk, Hq, Hk, d, 0) > G.GQA_NOALLOC_SCRATCH_BYTES
+    q, k, v = P.device_inputs(5004, *shp, on_device_gen=True)
+    out = torch.full((B, Sq, Hq, d), float("nan"), device="cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), device="cuda")
+    assert _noalloc(L, q, k, v, out, lse, shp, 0, -1, 0) == 0
+    torch.cuda.synchronize()
+    ref_out, ref_lse = G.gqa_attn_fwd(q, k, v, causal=0)
+    torch.cuda.synchronize()
+    assert (out - ref_out).abs().max().item() <= P.VARIANT_MAX
+    assert (lse - ref_lse).abs().max().item() <= P.VARIANT_MAX
+
+
+def test_noalloc_runs_split_calls_while_allocation_fails():
+    """With the library's allocation failure switch on (GQA_FAULT_INJECT_ALLOC, which
+    makes gqa_attn_fwd's split-KV allocation fail as on an exhausted device), a split
+    call of gqa_attn_fwd returns GQA_ERR_ALLOC while the allocation-free entry point runs
+    the same split and matches the unsplit result: it makes no allocation."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gqa_exact_attention_b200 as G
+    L = G.load()
+    shp = (4, 1, 4096, 32, 8, 128)
+    B, Sq, Sk, Hq, Hk, d = shp
+    q, k, v = P.device_inputs(5005, *shp)
+    ref_out, ref_lse = G.gqa_attn_fwd(q, k, v, causal=0, num_splits=1)
+    torch.cuda.synchronize()
+    out = torch.full((B, Sq, Hq, d), float("nan"), device="cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), device="cuda")
+    os.environ["GQA_FAULT_INJECT_ALLOC"] = "1"
+    try:
+        with pytest.raises(G.GqaError) as e:
+            G.gqa_attn_fwd(q, k, v, out=out, lse=lse, causal=0, num_splits=4)
+        assert e.value.status == 7  # GQA_ERR_ALLOC
+        assert _noalloc(L, q, k, v, out, lse, shp, 0, -1, 4) == 0
+        torch.cuda.synchronize()
+    finally:
+        del os.environ["GQA_FAULT_INJECT_ALLOC"]
+    assert (out - ref_out).abs().max().item() <= P.VARIANT_MAX
+    assert (lse - ref_lse).abs().max().item() <= P.VARIANT_MAX
