@@ -249,9 +249,26 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, c
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting or when
 // this wait ran past the time limit (then it records the timeout and starts the abort).
+// Normal limits: suspending probes (try_wait), the clock and the abort flag read every 256
+// of them.  Limits under 100 us exist only to exercise this path; a suspending probe can
+// cover a whole wait of several microseconds by itself, so those use non-suspending probes
+// (test_wait) and read the clock at every probe, and a wait of a few microseconds
+// reliably runs out.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile uint32_t* abort_flag,
                                              const FwdParams& p) {
+    if (p.timeout_ns < 100000) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_test_wait(bar, parity)) {
+            if (*abort_flag) return false;
+            if ((long long)(globaltimer() - t0) > p.timeout_ns) {
+                *abort_flag = 1u;
+                atomicOr(p.status ? p.status : &g_device_status, 1u);
+                return false;
+            }
+        }
+        return true;
+    }
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer();
     uint32_t spins = 0;
@@ -268,11 +285,13 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
     return true;
 }
 
-// Wait used during teardown: ignores the abort flag, gives up silently at the limit.
+// Wait used during teardown: ignores the abort flag, gives up silently at its own limit
+// (p.drain_ns, at least 1 s: copies and MMAs already issued finish in microseconds, and
+// they must land before the CTA's shared and tensor memory are released).
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const FwdParams& p) {
     uint64_t t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if ((long long)(globaltimer() - t0) > p.timeout_ns) return;
+        if ((long long)(globaltimer() - t0) > p.drain_ns) return;
     }
 }
 
@@ -645,7 +664,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 continue;
             }
 
-            float m = kNegInf;  // reference max of c*s (log2 units)
+            float m = 0.f;  // reference max of c*s (log2 units), see below
             float l = 0.f;
             for (int it = 0; it < n_t; ++it) {
                 ok = __all_sync(0xffffffffu, wait_bounded(s_full(t), sn & 1u, abort_flag, p));
@@ -714,18 +733,27 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                     e[0] = extremum([](float x, float y, float z) { return min3(x, y, z); },
                                     [](float x, float y) { return fminf(x, y); });
                 const float mx = (lim <= 0) ? kNegInf : (c == 0.f ? 0.f : e[0] * c);
-                // Deferred rescaling: move the reference max only when the block's max
-                // exceeds it by more than 8 (a factor 256), which keeps every p <= 256.
-                const bool grow = mx > m + 8.0f;  // false when mx = -inf; true when m = -inf < mx
+                // Reference max m (log2 units).  It starts at 0, not at the row's first
+                // block max, and moves only when a block's max leaves the window [m - 64,
+                // m + 8]: up past m + 8 (deferred rescaling, which keeps every p <= 256),
+                // or, while nothing has been summed yet, far below m (keys whose p would
+                // underflow).  It then moves to the block max rounded up to an integer.
+                // For scores within the window (typical attention logits) m stays 0 in every
+                // schedule, so x = c s is rounded once, the same way whether the key axis is
+                // split or the heads packed, and P is bit-identical across the scheduling
+                // variants; where m does move, it moves by integers, so p changes by exact
+                // powers of two and the rescale factors are exact.
+                const bool grow = mx > m + 8.0f || (l == 0.f && mx > kNegInf && mx < m - 64.f);
                 float alpha = 1.f;
                 if (grow) {
-                    alpha = (m == kNegInf) ? 0.f : ex2_approx(m - mx);
+                    const float m_new = ceilf(mx);
+                    alpha = (l == 0.f) ? 0.f : ex2_approx(m - m_new);  // nothing summed: O is 0
                     l *= alpha;
-                    m = mx;
+                    m = m_new;
                 }
                 // P = 2^(c*s - m) as bf16, written over S in TMEM (S is in registers).  A
                 // disallowed key gets the exponent -inf, i.e. p = 0, for any sign of c.
-                const float neg_m = (m == kNegInf) ? 0.f : -m;
+                const float neg_m = -m;
                 float ls0 = 0.f, ls1 = 0.f;
                 // the pairs of a chunk that take the polynomial, spread over the chunk
                 auto use_poly = [](int ch, int i) { return ((i * 5 + ch * 3) & 15) < C::kPolyPairs; };

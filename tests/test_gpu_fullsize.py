@@ -7,6 +7,11 @@ scheduler's own choice of pack/splits, as the benchmark runs it); the batch-size
 B in {16..256}, causal and not, with pack/split variants; decode Sq=1 against
 Sk in {2048, 8192, 32768} for B in {32, 128, 256} and splits in {1, 2, 4, 8}; and the
 long causal case Sq=Sk=16384, B=4, for d in {64, 128} and MHA/GQA/MQA head ratios.
+
+Scheduling variants (pack_gqa, num_splits) are also compared as whole tensors with the
+unsplit GPU run of the same inputs: out and lse within 1e-3 everywhere, in every cell of
+the batch sweep (B 16..256 x causal x 6 variants) and of the decode grid (splits 2/4/8
+and one q-head per tile against the unsplit packed run).
 """
 import numpy as np
 import pytest
@@ -63,27 +68,57 @@ def test_batch_sweep_heuristic(B, causal):
     run_sampled(1002 + B, (B, 2048, 2048, 32, 8, 128), causal)
 
 
-@pytest.mark.parametrize("B,causal", [(16, 0), (16, 1), (256, 1)])
+def max_abs_diff(a, b, chunk=16):
+    """max |a - b| over whole tensors, a batch slice at a time (no full-size temporary)."""
+    m = 0.0
+    for i in range(0, a.shape[0], chunk):
+        m = max(m, (a[i:i + chunk] - b[i:i + chunk]).abs().max().item())
+    return m
+
+
+def check_variants(seed, shp, causal, base, variants, n_rows):
+    """Each scheduling variant against the fp64 oracle on sampled rows, and as whole
+    tensors against the base schedule's GPU result: within 1e-3 everywhere (the
+    variants differ only in fp32 summation order)."""
+    import gqa_exact_attention_b200 as G
+    inp = P.device_inputs(seed, *shp, on_device_gen=True)
+    q, k, v = inp
+    run_sampled(seed, shp, causal, base[0], base[1], n_rows=n_rows, inputs=inp)
+    o_base, l_base = G.gqa_attn_fwd(q, k, v, causal=causal, pack_gqa=base[0], num_splits=base[1])
+    torch.cuda.synchronize()
+    worst = 0.0
+    for pack, splits in variants:
+        run_sampled(seed, shp, causal, pack, splits, n_rows=n_rows, inputs=inp)
+        o, l = G.gqa_attn_fwd(q, k, v, causal=causal, pack_gqa=pack, num_splits=splits)
+        torch.cuda.synchronize()
+        do, dl = max_abs_diff(o, o_base), max_abs_diff(l, l_base)
+        assert do <= P.VARIANT_MAX and dl <= P.VARIANT_MAX, (pack, splits, do, dl)
+        worst = max(worst, do, dl)
+        del o, l
+    del inp, o_base, l_base
+    torch.cuda.empty_cache()
+    return worst
+
+
+# the batch-size sweep: every B, causal and not, all six pack x split variants against
+# the unpacked unsplit run
+@pytest.mark.parametrize("B", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("causal", [0, 1])
 def test_batch_sweep_variants(B, causal):
     shp = (B, 2048, 2048, 32, 8, 128)
-    seed = 1102 + B + causal
-    inp = P.device_inputs(seed, *shp, on_device_gen=True)
-    for pack in (0, 1):
-        for splits in (1, 2, 4):
-            run_sampled(seed, shp, causal, pack, splits, n_rows=48, inputs=inp)
+    variants = [(pk, sp) for pk in (0, 1) for sp in (1, 2, 4) if (pk, sp) != (0, 1)]
+    check_variants(1102 + B + causal, shp, causal, (0, 1), variants, n_rows=48)
 
 
+# the decode grid: splits 1/2/4/8 with the heuristic's packing, and one q-head per tile,
+# each on sampled rows against the oracle; splits 2/4/8 and pack 0 as whole tensors
+# against the unsplit packed run
 @pytest.mark.parametrize("Sk", [2048, 8192, 32768])
 @pytest.mark.parametrize("B", [32, 128, 256])
 def test_decode(Sk, B):
     shp = (B, 1, Sk, 32, 8, 128)
     seed = 1003 + Sk + B
-    inp = P.device_inputs(seed, *shp, on_device_gen=True)
-    for splits in (1, 2, 4, 8):
-        run_sampled(seed, shp, 0, -1, splits, n_rows=16, inputs=inp)
-    run_sampled(seed, shp, 0, 0, 0, n_rows=16, inputs=inp)  # one q-head per tile
-    del inp
-    torch.cuda.empty_cache()
+    check_variants(seed, shp, 0, (1, 1), [(1, 2), (1, 4), (1, 8), (0, 1)], n_rows=16)
 
 
 @pytest.mark.parametrize("d", [64, 128])

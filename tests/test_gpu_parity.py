@@ -82,7 +82,11 @@ def test_empty_rows(pack, splits):
 
 
 # --- closed forms on the GPU: scale 0 gives the mean of V over the allowed keys;
-#     causal row 0 with Sq == Sk is v_0 exactly.
+#     causal row 0 with Sq == Sk sees one key: O = v_0 and LSE = scale q_0 . k_0.  The
+#     kernel keeps its reference max integral (so that every schedule rounds P alike), so
+#     the single weight is p = 2^(x - ceil(x)) in (1/2, 1]; the MMA takes p rounded to bf16
+#     while l keeps p, so O = v_0 * bf16(p) / p: within a relative 2^-8 of v_0 (the
+#     round-to-nearest bound of bf16's 8-bit significand), plus fp32 rounding.
 def test_scale_zero_and_single_key():
     shp = (1, 200, 200, 4, 2, 128)
     seed = 3100
@@ -95,7 +99,11 @@ def test_scale_zero_and_single_key():
     ln = torch.log(torch.arange(1, 201, device="cuda", dtype=torch.float32))
     assert (lse - ln.view(1, 1, -1)).abs().max().item() <= 1e-5
     out, lse = run(q, k, v, 1, 0, 1)
-    assert torch.equal(out[0, 0, 0], vf[0, 0, 0]) and torch.equal(out[0, 0, 3], vf[0, 0, 1])
+    for h, kvh in ((0, 0), (3, 1)):
+        v0 = vf[0, 0, kvh]
+        assert ((out[0, 0, h] - v0).abs() <= 2.0 ** -8 * 1.0001 * v0.abs() + 1e-30).all()
+        s0 = (q[0, 0, h].double() * k[0, 0, kvh].double()).sum().item() / 128 ** 0.5
+        assert abs(lse[0, h, 0].item() - s0) <= 1e-5 * max(1.0, abs(s0))
 
 
 # --- odd shapes / head ratios: Sq=77 vs Sk=4096 non-causal, d in {64,128},
