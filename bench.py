@@ -3,7 +3,13 @@
 
 Default workload: prefill GQA, B=64, Hq=32, Hk=8, Sq=Sk=2048, d=128, bf16 Q/K/V ~ N(0,1)
 (seeded, synthetic), causal, scale 1/sqrt(128), pack_gqa / num_splits from the heuristic.
-One step = one forward over the whole batch.  Rank 0 prints one JSON line.
+One step = one forward over the whole batch.  Rank 0 prints one JSON line.  Besides the
+headline (the step timed over --steps launches), the line carries:
+  "sustained"  the same step over a timed region of at least 1.2 s, against the sustained
+               GEMM peak (power and clocks settle over such a region);
+  "decode"     the metric's decode half: B=256, Sq=1, Sk=8192, Hq=32, Hk=8, d=128
+               (K and V 8.6 GB), device-timed like the headline, in HBM GB/s against
+               the measured copy bandwidth, with its own CPU-oracle baseline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -223,7 +229,10 @@ def oracle_sample(cfg, budget_s):
 
     # calibrate on one sequence restricted to a few heads' worth of time
     t1, threads = one(1, 0)
-    nb = max(1, min(B, int(budget_s / max(t1, 1e-3))))
+    nb = max(1, min(B - 1 if B > 1 else 1, int(budget_s / max(t1, 1e-3))))
+    # keep the fp64 copies of the sample within about 1 GB per tensor
+    per_seq = max(Sq * Hq * d, Sk * Hk * d)
+    nb = max(1, min(nb, (1 << 27) // per_seq))
     if nb > 1:
         tn, threads = one(nb, 1)
         total_t, total_b = t1 + tn, 1 + nb
@@ -236,6 +245,84 @@ def oracle_sample(cfg, budget_s):
 
 
 # ----------------------------------------------------------------- GPU arm
+
+# The decode half of the metric: one new query token per sequence against its keys,
+# B=256, Sk=8192 (K and V 8.6 GB, far above the 126 MB L2), Hq=32, Hk=8, d=128,
+# non-causal, pack_gqa / num_splits from the heuristic.
+DECODE_CFG = {"name": "decode B=256 Hq=32 Hk=8 Sq=1 Sk=8192 d=128 non-causal", "B": 256,
+              "Sq": 1, "Sk": 8192, "Hq": 32, "Hk": 8, "d": 128, "causal": 0, "seed": 1003,
+              "l2": "inputs larger than L2 (K and V 8590 MB read per step)"}
+
+
+def time_steps(step, steps, stream, per_launch=True):
+    """Time `steps` calls of step() on `stream` with CUDA events: (total ms, mean ms of
+    one call measured by its own event pair)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps if per_launch else 0)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(steps):
+        if per_launch:
+            ev[i][0].record(stream)
+        step()
+        if per_launch:
+            ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    total = t_start.elapsed_time(t_end)
+    mean = statistics.mean(a.elapsed_time(b) for a, b in ev) if per_launch else total / steps
+    return total, mean
+
+
+def run_decode(args, pg, world, rank, dev, peaks, peak_src):
+    """The decode workload, device-timed like the main step: the 'decode' object of the
+    JSON line (HBM GB/s against the measured copy bandwidth)."""
+    import torch
+
+    import gqa_exact_attention_b200 as G
+    import inputs
+    c = DECODE_CFG
+    B, Sq, Sk, Hq, Hk, d = (c[k] for k in ("B", "Sq", "Sk", "Hq", "Hk", "d"))
+    pack, splits = G.gqa_attn_choose(B, Sq, Sk, Hq, Hk, d, 0)
+    seed = c["seed"] + rank
+    q = inputs.device_tensor(seed, inputs.TID_Q, (B, Sq, Hq, d), device=dev)
+    k = inputs.device_tensor(seed, inputs.TID_K, (B, Sk, Hk, d), device=dev)
+    v = inputs.device_tensor(seed, inputs.TID_V, (B, Sk, Hk, d), device=dev)
+    out = torch.empty((B, Sq, Hq, d), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        G.gqa_attn_fwd(q, k, v, out=out, lse=lse, causal=0, pack_gqa=pack, num_splits=splits,
+                       stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(pg)
+    torch.cuda.synchronize()
+    total_ms, launch_ms = time_steps(step, args.steps, stream)
+    barrier(pg)
+    total_ms = max_over_ranks(pg, total_ms)
+    launch_ms = max_over_ranks(pg, launch_ms)
+    by = hbm_bytes(B, Sq, Sk, Hq, Hk, d)
+    achieved = by / (launch_ms / 1e3) / 1e9
+    obj = {
+        "workload": c["name"], "value": round(job_throughput(by, world, total_ms, args.steps) / 1e9, 1),
+        "unit": "GB/s", "ms_per_step": round(total_ms / args.steps, 4), "steps": args.steps,
+        "tokens_per_s": round(world * B / (total_ms / args.steps / 1e3), 1),
+        "pack_gqa": pack, "num_splits": splits, "l2": c["l2"],
+        "gpu_launches": (1 + (1 if splits > 1 else 0)) * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "peak_source": f"{peak_src}:hbm_gbs",
+                     "traffic": traffic_for(c["name"], pack, splits), "kernel": "gqa_fwd_kernel"},
+    }
+    del q, k, v, out, lse
+    torch.cuda.empty_cache()
+    return obj
+
 
 def run_gpu(args, cfg):
     import torch
@@ -274,24 +361,24 @@ def run_gpu(args, cfg):
     torch.cuda.synchronize()
 
     # ---- device-timed region: K steps, events per launch on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
     barrier(pg)
     torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    t_end.record(stream)
-    torch.cuda.synchronize()
+    total_ms, launch_ms = time_steps(step, args.steps, stream)
     barrier(pg)
-    total_ms = max_over_ranks(pg, t_start.elapsed_time(t_end))
-    launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    total_ms = max_over_ranks(pg, total_ms)
     launch_ms = max_over_ranks(pg, launch_ms)
     ms_per_step = total_ms / args.steps
+
+    # ---- the same step over a timed region of at least a second (power and clocks
+    # settle), reported against the sustained GEMM peak
+    sus_steps = 0
+    if not args.no_sustained:
+        sus_steps = max(args.steps, min(4000, int(math.ceil(1200.0 / max(ms_per_step, 1e-3)))))
+        barrier(pg)
+        torch.cuda.synchronize()
+        sus_total, _ = time_steps(step, sus_steps, stream, per_launch=False)
+        barrier(pg)
+        sus_total = max_over_ranks(pg, sus_total)
     if G.gqa_attn_device_status(reset=True) != 0:
         raise SystemExit("an in-kernel bounded wait timed out during the benchmark")
 
@@ -358,11 +445,14 @@ def run_gpu(args, cfg):
     barrier(pg)
     e2e_ms = max_over_ranks(pg, e0.elapsed_time(e1)) / e_steps
     del bufs
+    peaks, peak_src = load_peaks()
+    decode = None
+    if cfg.get("with_decode"):
+        decode = run_decode(args, pg, world, rank, dev, peaks, peak_src)
     clocks = sampler.stop() if sampler else None
 
     fl = flops(B, Sq, Sk, Hq, d, causal)
     by = hbm_bytes(B, Sq, Sk, Hq, Hk, d)
-    peaks, peak_src = load_peaks()
     decode_like = Sq * (Hq // Hk) <= 128 and not causal
     timed_s = total_ms / 1e3
     if decode_like:
@@ -405,6 +495,19 @@ def run_gpu(args, cfg):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if sus_steps and not decode_like:
+        sus_ms = sus_total / sus_steps
+        sus_val = job_throughput(fl, world, sus_total, sus_steps) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        line["sustained"] = {
+            "value": round(sus_val, 3), "unit": unit, "steps": sus_steps,
+            "timed_s": round(sus_total / 1e3, 3), "ms_per_step": round(sus_ms, 4),
+            "gpu_launches": launches_per_step * sus_steps,
+            "roofline": {"bound": "tensor", "achieved": fl / (sus_ms / 1e3) / 1e12, "peak": pk,
+                         "unit": "TFLOP/s", "frac": fl / (sus_ms / 1e3) / 1e12 / pk,
+                         "peak_source": f"{peak_src}:bf16_tflops_sustained"}}
+    if decode is not None:
+        line["decode"] = decode
     if rank == 0 and not args.no_cpu_baseline:
         rate, threads, desc = oracle_sample(cfg, args.cpu_budget)
         if decode_like:
@@ -413,6 +516,13 @@ def run_gpu(args, cfg):
             cv = rate / 1e12
         line["cpu_baseline"] = {"value": cv, "unit": unit, "cores": threads, "kind": "oracle",
                                 "sample": desc}
+        if decode is not None:
+            dc = DECODE_CFG
+            drate, dthreads, ddesc = oracle_sample(dc, min(args.cpu_budget, 8.0))
+            dfl = flops(dc["B"], dc["Sq"], dc["Sk"], dc["Hq"], dc["d"], 0)
+            dby = hbm_bytes(dc["B"], dc["Sq"], dc["Sk"], dc["Hq"], dc["Hk"], dc["d"])
+            decode["cpu_baseline"] = {"value": dby / (dfl / drate) / 1e9, "unit": "GB/s",
+                                      "cores": dthreads, "kind": "oracle", "sample": ddesc}
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
@@ -592,6 +702,10 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="skip the >= 1 s timed region of the main step")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode workload of the default line")
     ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache"], default=None,
                     help="print one line per configuration of the batch sweep or decode grid")
     args = ap.parse_args()
@@ -604,6 +718,7 @@ def main():
     in_bytes = 2 * (args.B * args.Sq * args.Hq * args.d + 2 * args.B * args.Sk * args.Hk * args.d)
     cfg = {"name": name, "B": args.B, "Sq": args.Sq, "Sk": args.Sk, "Hq": args.Hq, "Hk": args.Hk,
            "d": args.d, "causal": args.causal, "seed": 1001,
+           "with_decode": default and not args.no_decode,
            "l2": (f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB read per step)"
                   if in_bytes > 126e6 else f"inputs {in_bytes / 1e6:.1f} MB, L2-resident")}
     if args.impl == "reference":
