@@ -15,9 +15,9 @@ headline (the step timed over --steps launches), the line carries:
 
 --impl reference times the fp64 CPU oracle (the only reference this project has) on the
 box's host cores, on bounded samples of the same workload.  Other flags (--B, --Sq, ...)
-select another shape for ad-hoc measurement; ``--sweep prefill|decode|kvcache`` prints one line
-per configuration of the batch-sensitivity sweep, the decode grid, or the KV-cache entry
-point (per-sequence lengths, bf16 output).
+select another shape for ad-hoc measurement; ``--sweep prefill|decode|kvcache|paged`` prints
+one line per configuration of the batch-sensitivity sweep, the decode grid, the KV-cache
+entry point (per-sequence lengths, bf16 output), or the paged KV cache next to the dense one.
 """
 from __future__ import annotations
 
@@ -580,6 +580,8 @@ def run_sweep(args):
     peaks, _ = load_peaks()
     if args.sweep == "kvcache":
         return run_sweep_kvcache(args, peaks)
+    if args.sweep == "paged":
+        return run_sweep_paged(args, peaks)
     if args.sweep == "prefill":
         cases = [(B, 2048, 2048, c, pk, sp) for B in (16, 32, 64, 128, 256) for c in (1, 0)
                  for (pk, sp) in [(-1, 0), (0, 1), (1, 1), (0, 2), (1, 2), (0, 4), (1, 4)]]
@@ -685,6 +687,71 @@ def run_sweep_kvcache(args, peaks):
         torch.cuda.empty_cache()
 
 
+def run_sweep_paged(args, peaks):
+    """Kernel-only timings of gqa_attn_fwd_paged next to gqa_attn_fwd_kvcache on the same
+    keys: decode against a capacity of 8192 keys per sequence, seeded lengths uniform in
+    [1, 8192] (B 32/128/256), automatic schedule, fp32 output; page sizes 16, 64 and 256,
+    pages handed out in a shuffled order.  Bytes count each sequence's own keys."""
+    import numpy as np
+    import torch
+
+    import gqa_exact_attention_b200 as G
+    import inputs
+    stream = torch.cuda.current_stream()
+    Hq, Hk, d, cap, Sq = 32, 8, 128, 8192, 1
+
+    def timed(step):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if G.gqa_attn_device_status(reset=True) != 0:
+            raise SystemExit("an in-kernel bounded wait timed out")
+        return e0.elapsed_time(e1) / args.steps
+
+    for B in (32, 128, 256):
+        rng = np.random.default_rng(7000 + B)
+        lens = rng.integers(1, cap + 1, size=B)
+        sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        q = inputs.device_tensor(1001, inputs.TID_Q, (B, Sq, Hq, d))
+        out = torch.empty((B, Sq, Hq, d), dtype=torch.float32, device="cuda")
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
+        keys = int(lens.sum())
+        by = 2 * B * Sq * Hq * d + 2 * 2 * keys * Hk * d + 4 * B * Sq * Hq * d + 4 * B * Hq * Sq
+        k = inputs.device_tensor(1001, inputs.TID_K, (B, cap, Hk, d))
+        v = inputs.device_tensor(1001, inputs.TID_V, (B, cap, Hk, d))
+        ms_dense = timed(lambda: G.gqa_attn_fwd_kvcache(q, k, v, sl, out=out, lse=lse, stream=stream))
+        del k, v
+        torch.cuda.empty_cache()
+        for ps in (16, 64, 256):
+            need = (lens + ps - 1) // ps
+            num_pages = int(need.sum())
+            perm = rng.permutation(num_pages)
+            table = np.zeros((B, cap // ps), dtype=np.int32)
+            o = 0
+            for b in range(B):
+                table[b, :need[b]] = perm[o:o + need[b]]
+                o += need[b]
+            tt = torch.from_numpy(table).cuda()
+            kp = inputs.device_tensor(1002, inputs.TID_K, (num_pages, ps, Hk, d))
+            vp = inputs.device_tensor(1002, inputs.TID_V, (num_pages, ps, Hk, d))
+            ms = timed(lambda: G.gqa_attn_fwd_paged(q, kp, vp, tt, sl, out=out, lse=lse, stream=stream))
+            print(json.dumps({"sweep": "paged", "B": B, "Sk_capacity": cap, "page_size": ps,
+                              "mean_length": round(float(lens.mean()), 1), "ms": round(ms, 4),
+                              "hbm_gbs": round(by / ms / 1e6, 1),
+                              "frac_of_measured_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 3),
+                              "dense_kvcache_ms": round(ms_dense, 4),
+                              "dense_kvcache_gbs": round(by / ms_dense / 1e6, 1),
+                              "paged_over_dense": round(ms_dense / ms, 3)}), flush=True)
+            del kp, vp
+            torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -706,7 +773,7 @@ def main():
                     help="skip the >= 1 s timed region of the main step")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode workload of the default line")
-    ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache"], default=None,
+    ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache", "paged"], default=None,
                     help="print one line per configuration of the batch sweep or decode grid")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -15,7 +15,8 @@ import os
 
 __all__ = [
     "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes", "gqa_attn_status_string",
-    "gqa_attn_device_status", "gqa_attn_fwd_noalloc", "GqaError", "lib_path", "load",
+    "gqa_attn_device_status", "gqa_attn_fwd_noalloc", "gqa_attn_fwd_kvcache",
+    "gqa_attn_fwd_paged", "GqaError", "lib_path", "load",
     "GQA_NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -74,6 +75,8 @@ def load():
     L.gqa_attn_fwd_noalloc.restype = i
     L.gqa_attn_fwd_kvcache.argtypes = [p, p, p, p, p, i, p, i, i, i, i, i, i, f, i, i, i, p]
     L.gqa_attn_fwd_kvcache.restype = i
+    L.gqa_attn_fwd_paged.argtypes = [p, p, p, p, i, p, i, i, p, i, p, i, i, i, i, i, f, i, i, i, p]
+    L.gqa_attn_fwd_paged.restype = i
     _lib = L
     return L
 
@@ -212,4 +215,53 @@ def gqa_attn_fwd_kvcache(q, k_cache, v_cache, cache_seqlens=None, out=None, lse=
             None if cache_seqlens is None else cache_seqlens.data_ptr(), out.data_ptr(), code,
             lse.data_ptr(), B, Sq, Sk, Hq, Hk, d, float(scale), int(bool(causal)),
             int(pack_gqa), int(num_splits), stream.cuda_stream))
+    return out, lse
+
+
+def gqa_attn_fwd_paged(q, k_pages, v_pages, block_table, cache_seqlens, out=None, lse=None,
+                       out_dtype=None, scale=None, causal=False, pack_gqa=-1, num_splits=0,
+                       stream=None):
+    """out, lse = gqa_attn_fwd_paged(q, k_pages, v_pages, block_table, cache_seqlens, ...).
+
+    k_pages, v_pages: bf16 [num_pages, page_size, Hk, d] page pools; block_table: int32
+    CUDA tensor [B, max_pages_per_seq] (key j of sequence b is row j % page_size of page
+    block_table[b, j // page_size]); cache_seqlens: int32 CUDA tensor [B].  out is fp32 or
+    bf16 [B, Sq, Hq, d]; lse fp32 [B, Hq, Sq].  Causal masks are bottom-right aligned to
+    each sequence's own length.
+    """
+    import torch
+
+    B, Sq, Hq, d = q.shape
+    num_pages, page_size, Hk = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if k_pages.shape != v_pages.shape or k_pages.shape[3] != d:
+        raise ValueError("k_pages and v_pages must be [num_pages, page_size, Hk, d] matching q")
+    for name, t in (("block_table", block_table), ("cache_seqlens", cache_seqlens)):
+        if t.dtype != torch.int32 or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{name} must be a contiguous int32 tensor on q's device")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(cache_seqlens.shape) != (B,):
+        raise ValueError("block_table must be [B, max_pages_per_seq] and cache_seqlens [B]")
+    if out is None:
+        dt = torch.float32 if out_dtype is None else out_dtype
+        out = torch.empty((B, Sq, Hq, d), dtype=dt, device=q.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or not out.is_contiguous() \
+            or out.device != q.device or tuple(out.shape) != (B, Sq, Hq, d):
+        raise ValueError("out must be a contiguous fp32 or bf16 tensor [B, Sq, Hq, d] on q's device")
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("lse must be a contiguous fp32 tensor [B, Hq, Sq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    code = GQA_OUT_BF16 if out.dtype == torch.bfloat16 else GQA_OUT_F32
+    with torch.cuda.device(q.device):
+        _check(load().gqa_attn_fwd_paged(
+            q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+            int(block_table.shape[1]), cache_seqlens.data_ptr(), num_pages, page_size,
+            out.data_ptr(), code, lse.data_ptr(), B, Sq, Hq, Hk, d, float(scale),
+            int(bool(causal)), int(pack_gqa), int(num_splits), stream.cuda_stream))
     return out, lse

@@ -379,16 +379,36 @@ size_t partial_bytes(int splits, int B, int Sq, int Hq, int d) {
     return (size_t)splits * (size_t)B * Hq * Sq * ((size_t)d + 1) * sizeof(float);
 }
 
+// A paged KV cache: k and v are page pools [num_pages, page_size, Hk, d]; key j of
+// sequence b is row j % page_size of page block_table[b * table_stride + j / page_size].
+struct Paged {
+    const int* block_table = nullptr;
+    int table_stride = 0;
+    int page_size = 0;
+    int num_pages = 0;
+};
+
+bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
+
 // The forward behind every entry point.  out is fp32 or, with out_bf16, bf16; seqlens_k
 // (device, nullable) gives each sequence's key count; fixed (nullable) replaces the pool
-// allocation of the split partials.
+// allocation of the split partials; paged (nullable) makes k and v page pools.
 gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seqlens_k, void* out,
                     bool out_bf16, float* lse, int B, int Sq, int Sk, int Hq, int Hk, int d,
                     float scale, int causal, int pack_gqa, int num_splits, void* stream_ptr,
-                    const Scratch* fixed = nullptr) {
+                    const Scratch* fixed = nullptr, const Paged* paged = nullptr) {
     if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
-    gqa_status st = validate_shape(B, Sq, Sk, Hq, Hk, d, pack_gqa, num_splits);
+    // a paged cache's logical capacity is not a dense tensor: its pool is checked below
+    gqa_status st = validate_shape(B, Sq, paged ? 1 : Sk, Hq, Hk, d, pack_gqa, num_splits);
     if (st != GQA_OK) return st;
+    if (paged != nullptr) {
+        if (!paged->block_table || !seqlens_k) return GQA_ERR_NULL;
+        if (!is_pow2(paged->page_size) || paged->page_size < 16 || paged->num_pages < 1 ||
+            paged->table_stride < 1 ||
+            (long long)paged->num_pages * paged->page_size * Hk >= (1ll << 31))
+            return GQA_ERR_SHAPE;
+        if ((reinterpret_cast<uintptr_t>(paged->block_table) & 3u) != 0) return GQA_ERR_ALIGN;
+    }
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
         return GQA_ERR_ALIGN;
     if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) != 0) return GQA_ERR_ALIGN;
@@ -417,10 +437,26 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     const int g = Hq / Hk;
 
     gqa::FwdParams p{};
-    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM) ||
-        !encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
-        !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
+    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM))
         return GQA_ERR_CUDA;
+    if (paged == nullptr) {
+        if (!encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
+            !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
+            return GQA_ERR_CUDA;
+    } else {
+        // the page pools as (d, Hk, page_size, num_pages), boxes of up to 128 rows
+        const int rows = paged->page_size < kBlockN ? paged->page_size : kBlockN;
+        if (!encode_bshd(&p.tm_k, k, paged->num_pages, paged->page_size, Hk, d, 1, rows) ||
+            !encode_bshd(&p.tm_v, v, paged->num_pages, paged->page_size, Hk, d, 1, rows))
+            return GQA_ERR_CUDA;
+        p.block_table = paged->block_table;
+        p.table_stride = paged->table_stride;
+        int shift = 0;
+        while ((1 << shift) < paged->page_size) ++shift;
+        p.page_shift = shift;
+        p.page_rows = rows;
+        p.num_pages = paged->num_pages;
+    }
     p.out = out_bf16 ? nullptr : static_cast<float*>(out);
     p.out_bf16 = out_bf16 ? static_cast<uint16_t*>(out) : nullptr;
     p.seqlens_k = seqlens_k;
@@ -553,6 +589,25 @@ gqa_status gqa_attn_fwd_kvcache(const void* q, const void* k_cache, const void* 
     if (out_dtype != GQA_OUT_F32 && out_dtype != GQA_OUT_BF16) return GQA_ERR_SHAPE;
     return fwd_impl(q, k_cache, v_cache, cache_seqlens, out, out_dtype == GQA_OUT_BF16, lse, B,
                     Sq, Sk, Hq, Hk, d, scale, causal, pack_gqa, num_splits, stream);
+}
+
+gqa_status gqa_attn_fwd_paged(const void* q, const void* k_pages, const void* v_pages,
+                              const int* block_table, int max_pages_per_seq,
+                              const int* cache_seqlens, int num_pages, int page_size, void* out,
+                              int out_dtype, float* lse, int B, int Sq, int Hq, int Hk, int d,
+                              float scale, int causal, int pack_gqa, int num_splits, void* stream) {
+    if (out_dtype != GQA_OUT_F32 && out_dtype != GQA_OUT_BF16) return GQA_ERR_SHAPE;
+    if (max_pages_per_seq < 1 || page_size < 1 ||
+        (long long)max_pages_per_seq * page_size >= (1ll << 31))
+        return GQA_ERR_SHAPE;
+    Paged pg;
+    pg.block_table = block_table;
+    pg.table_stride = max_pages_per_seq;
+    pg.page_size = page_size;
+    pg.num_pages = num_pages;
+    return fwd_impl(q, k_pages, v_pages, cache_seqlens, out, out_dtype == GQA_OUT_BF16, lse, B,
+                    Sq, max_pages_per_seq * page_size, Hq, Hk, d, scale, causal, pack_gqa,
+                    num_splits, stream, nullptr, &pg);
 }
 
 gqa_status gqa_attn_device_status(int reset) {

@@ -52,6 +52,15 @@ struct FwdParams {
     // bf16 output [B, Sq, Hq, d] instead of out (num_splits == 1; with splits the combine
     // writes it); NULL: fp32 out.  tm_o then maps it as bf16 with 64-column boxes.
     uint16_t* out_bf16;
+    // Paged KV cache (NULL block_table: dense k/v).  tm_k / tm_v then map the page pools
+    // [num_pages, page_size, Hk, d] as (d, Hk, page_size, num_pages) with boxes of
+    // page_rows = min(page_size, 128) rows; key j of sequence b lies in page
+    // block_table[b * table_stride + j / page_size], row j % page_size.
+    const int* block_table;
+    int table_stride;  // entries per sequence (pages per sequence at most)
+    int page_shift;    // log2(page_size)
+    int page_rows;     // rows of one TMA box: min(page_size, 128)
+    int num_pages;     // pages in the pool (a page coordinate past it reads zeros)
 };
 
 struct CombineParams {

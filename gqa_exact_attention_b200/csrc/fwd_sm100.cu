@@ -247,6 +247,33 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, c
     if (rm.ok) *lrow = lse_v;
 }
 
+// Paged KV: the block-table entries of one sequence, cached in the producer warp's
+// registers 32 at a time (lane i holds entry base + i), with the next 32 already loaded
+// (lane i of w1 holds base + 32 + i) so that moving on does not wait for memory.
+// Warp-collective: every lane calls it with the same arguments.
+struct PageCache {
+    int b = -1;
+    int base = 0;
+    int w0 = -1, w1 = -1;
+};
+__device__ __forceinline__ int table_entry(const FwdParams& p, int b, int i) {
+    return (i < p.table_stride) ? __ldg(p.block_table + (size_t)b * p.table_stride + i) : -1;
+}
+__device__ __forceinline__ int page_of(PageCache& pc, const FwdParams& p, int b, int page_i,
+                                       int lane) {
+    if (b != pc.b || page_i < pc.base || page_i >= pc.base + 64) {
+        pc.b = b;
+        pc.base = page_i & ~31;
+        pc.w0 = table_entry(p, b, pc.base + lane);
+        pc.w1 = table_entry(p, b, pc.base + 32 + lane);
+    } else if (page_i >= pc.base + 32) {
+        pc.base += 32;
+        pc.w0 = pc.w1;
+        pc.w1 = table_entry(p, b, pc.base + 32 + lane);
+    }
+    return __shfl_sync(0xffffffffu, pc.w0, page_i - pc.base);
+}
+
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting or when
 // this wait ran past the time limit (then it records the timeout and starts the abort).
 // Normal limits: suspending probes (try_wait), the clock and the abort flag read every 256
@@ -375,6 +402,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
             uint32_t ld = 0;       // K/V ring loads issued (K and V each count one)
             uint32_t qn[NT] = {};  // Q loads issued per tile
             bool ok = true;
+            PageCache pcache;      // paged KV only
             // Q_t of a unit, once the previous unit's last S_t has read the buffer
             auto load_q = [&](const UnitGeom<NT>& g, int t) {
                 if (g.n[t] == 0 || !ok) return;
@@ -401,6 +429,22 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 load_q(g, 0);
                 for (int it = 0; it < g.nblk && ok; ++it) {
                     const int kpos = (g.kb_lo + it) * kBlockN;
+                    // paged KV: the block's 128 keys come from 128 / page_rows pages (one
+                    // page row range each); sub-ranges at or past this sequence's key count
+                    // take a page coordinate past the pool, which TMA fills with zeros
+                    // (masked anyway), so no table entry past the sequence is used
+                    int pg[8], prow[8];
+                    const int nsub = p.block_table ? kBlockN / p.page_rows : 1;
+                    if (p.block_table) {
+#pragma unroll
+                        for (int sub = 0; sub < 8; ++sub) {
+                            if (sub >= nsub) break;
+                            const int key0 = kpos + sub * p.page_rows;
+                            const int page = page_of(pcache, p, g.b, key0 >> p.page_shift, lane);
+                            pg[sub] = key0 < g.sk ? page : p.num_pages;
+                            prow[sub] = key0 & ((1 << p.page_shift) - 1);
+                        }
+                    }
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
                         const int slot = ld % C::kSlots;
@@ -409,11 +453,23 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                         if (!ok) break;
                         if (elect_one()) {
                             mbar_arrive_expect_tx(kv_full(slot), (uint32_t)C::kTileBytes);
+                            const void* tm = w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v;
+                            if (p.block_table == nullptr) {
 #pragma unroll
-                            for (int c = 0; c < C::kChunks; ++c)
-                                tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes,
-                                            w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v,
-                                            kv_full(slot), c * 64, g.kvh, kpos, g.b);
+                                for (int c = 0; c < C::kChunks; ++c)
+                                    tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, tm,
+                                                kv_full(slot), c * 64, g.kvh, kpos, g.b);
+                            } else {
+#pragma unroll
+                                for (int sub = 0; sub < 8; ++sub) {
+                                    if (sub >= nsub) break;
+#pragma unroll
+                                    for (int c = 0; c < C::kChunks; ++c)
+                                        tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes +
+                                                        sub * p.page_rows * 128,
+                                                    tm, kv_full(slot), c * 64, g.kvh, prow[sub], pg[sub]);
+                                }
+                            }
                         }
                         __syncwarp();
                         ++ld;

@@ -181,6 +181,45 @@ GQA_API gqa_status gqa_attn_fwd_kvcache(const void* q, const void* k_cache, cons
                                         float scale, int causal, int pack_gqa, int num_splits,
                                         void* stream);
 
+/*
+ * gqa_attn_fwd_paged — the forward of gqa_attn_fwd_kvcache against a paged KV cache: the
+ * keys and values of every sequence live in fixed-size pages of a shared pool, found
+ * through a block table, instead of one dense [B, Sk, Hk, d] slab.
+ *
+ * The pages name a paged KV cache for sequences of changing length ("解锁Stable Diffusion
+ * 效率瓶颈…", section "行业应用场景拓展", scenario one: 分页KV缓存) and as the remedy when
+ * memory runs out for sequences longer than 8192 ("解锁Stable Diffusion效率瓶颈…", section
+ * "常见问题排查流程图", item 2 "内存溢出").
+ *
+ *   k_pages, v_pages   bf16 [num_pages, page_size, Hk, d], row-major, 16-byte aligned: the
+ *                      page pools.
+ *   block_table        device int32 [B, max_pages_per_seq], 4-byte aligned.  Key j of
+ *                      sequence b is row j % page_size of page
+ *                      block_table[b * max_pages_per_seq + j / page_size].  Only the entries
+ *                      of pages that hold a key j < L_b are used; an entry outside
+ *                      [0, num_pages) reads as a page of zeros (no fault).
+ *   cache_seqlens      device int32 [B], required.  Sequence b has L_b keys, L_b =
+ *                      cache_seqlens[b] clamped to [0, max_pages_per_seq * page_size].
+ *   page_size          a power of two >= 16 (e.g. 16, 64, 256).
+ *   other arguments    as gqa_attn_fwd_kvcache, with Sk = max_pages_per_seq * page_size.
+ *
+ * The keys of a page past L_b but in the page that holds key L_b - 1 are read by the
+ * kernel (masked out of the result); like the dense cache's rows past L_b, they must hold
+ * finite values.  Read on the device in stream order; the table and lengths must stay
+ * valid until the call's work on the stream is done.
+ *
+ * Errors as gqa_attn_fwd_kvcache; GQA_ERR_NULL for a NULL block_table or cache_seqlens;
+ * GQA_ERR_SHAPE for a page_size that is not a power of two >= 16, num_pages or
+ * max_pages_per_seq < 1, or a pool with 2^31 rows or more; GQA_ERR_ALIGN for a
+ * misaligned block_table.
+ */
+GQA_API gqa_status gqa_attn_fwd_paged(const void* q, const void* k_pages, const void* v_pages,
+                                      const int* block_table, int max_pages_per_seq,
+                                      const int* cache_seqlens, int num_pages, int page_size,
+                                      void* out, int out_dtype, float* lse, int B, int Sq, int Hq,
+                                      int Hk, int d, float scale, int causal, int pack_gqa,
+                                      int num_splits, void* stream);
+
 /* Static description of a status code. */
 GQA_API const char* gqa_attn_status_string(gqa_status status);
 

@@ -22,7 +22,7 @@ def test_header_declares_the_entry_points():
     assert declared_symbols() == sorted([
         "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes",
         "gqa_attn_status_string", "gqa_attn_device_status", "gqa_attn_fwd_noalloc",
-        "gqa_attn_fwd_kvcache"])
+        "gqa_attn_fwd_kvcache", "gqa_attn_fwd_paged"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -90,6 +90,28 @@ def test_kvcache_invalid_arguments(kw, code):
     assert kvcache_raw(**kw) == code
 
 
+def paged_raw(q=16, kp=16, vp=16, table=16, max_pages=4, seqlens=32, num_pages=8, page_size=16,
+              out=16, out_dtype=0, lse=16, B=1, Sq=8, Hq=4, Hk=2, d=64, scale=0.125, causal=0,
+              pack=-1, splits=0):
+    L = G.load()
+    return L.gqa_attn_fwd_paged(q, kp, vp, table, max_pages, seqlens, num_pages, page_size, out,
+                                out_dtype, lse, B, Sq, Hq, Hk, d, scale, causal, pack, splits, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(out_dtype=2), 2), (dict(max_pages=0), 2), (dict(page_size=0), 2),
+    (dict(page_size=8), 2), (dict(page_size=24), 2), (dict(page_size=96), 2), (dict(num_pages=0), 2),
+    (dict(table=NULL), 1), (dict(seqlens=NULL), 1), (dict(kp=NULL), 1), (dict(out=NULL), 1),
+    (dict(table=18), 5), (dict(kp=24), 5), (dict(seqlens=34), 5),
+    (dict(Hq=6, Hk=4), 3), (dict(d=96), 4), (dict(B=0), 2),
+    (dict(max_pages=1 << 20, page_size=1 << 12), 2),
+    (dict(num_pages=1 << 20, page_size=1 << 10, Hk=4, Hq=4), 2),
+])
+def test_paged_invalid_arguments(kw, code):
+    # fake pointers: every check happens on the host before anything is launched or read
+    assert paged_raw(**kw) == code
+
+
 def test_pages_head_constraint_example():
     """Hq must be a multiple of Hk (the pages' interface constraint); Hq=6, Hk=2 is valid."""
     L = G.load()
@@ -152,3 +174,4 @@ def test_no_gpu_is_an_error_not_a_fallback():
     assert kvcache_raw(seqlens=32, out_dtype=1) in (6, 8)
     L = G.load()
     assert L.gqa_attn_fwd_noalloc(16, 16, 16, 16, 16, 1, 8, 8, 4, 2, 64, 0.125, 0, -1, 0, None) in (6, 8)
+    assert paged_raw() in (6, 8)
