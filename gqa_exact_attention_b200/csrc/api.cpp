@@ -111,15 +111,17 @@ int choose_splits(const Plan& pl, int d, int num_sms) {
 
 // With per-sequence KV lengths the units' work varies from nothing to the capacity, and
 // the plan cannot see the lengths (they live on the device).  Split until there are at
-// least kVarlenUnitsPerSlot units per CTA slot: a slot then sums several units of
-// unrelated length, and the longest sequence is cut into that many pieces.  Never fewer
-// splits than the dense model picks for the capacity.
+// least kVarlenUnitsPerSlot units per CTA slot: the device-side work order then deals
+// them heaviest first over the CTAs (one-tile kernel), and a slot sums several units of
+// unrelated length.  The prefill kernel keeps its own order, so it also takes at least
+// the dense model's count for the capacity.
 int choose_splits_varlen(const Plan& pl, int d, int num_sms) {
     constexpr long long kVarlenUnitsPerSlot = 3;  // fitted on B200: uniform lengths, B 32-256
     const long long slots = (long long)num_sms * gqa::fwd_ctas_per_sm(d, pl.nt);
     const int smax = pl.kv_blocks < kMaxSplits ? pl.kv_blocks : kMaxSplits;
     int s = 1;
     while (s < smax && pl.units * s < kVarlenUnitsPerSlot * slots) ++s;
+    if (pl.nt == 1) return s;
     const int dense = choose_splits(pl, d, num_sms);
     return s > dense ? s : dense;
 }
@@ -484,26 +486,37 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     p.timeout_ns = timeout_ns();
     p.drain_ns = drain_ns(p.timeout_ns);
 
+    // Device scratch: the split partials (num_splits > 1), and with per-sequence lengths the
+    // work order of the units (2 ints per unit), in one stream-ordered pool allocation, or
+    // the caller's fixed scratch (which never comes with lengths).
     void* ws = nullptr;  // pool allocation to release after the combine (never with fixed)
-    if (pl.splits > 1) {
-        const size_t rows = (size_t)B * Hq * Sq;
-        const size_t bytes = partial_bytes(pl.splits, B, Sq, Hq, d);
-        void* part = nullptr;
+    const size_t rows = (size_t)B * Hq * Sq;
+    const size_t part_bytes = pl.splits > 1 ? (partial_bytes(pl.splits, B, Sq, Hq, d) + 255) & ~(size_t)255 : 0;
+    // (the one-tile kernel only: its units share no K/V, while the prefill kernel's unit
+    // order keeps a batch window's K/V in L2)
+    const size_t order_bytes =
+        (seqlens_k != nullptr && pl.nt == 1) ? 2 * (size_t)pl.units * sizeof(int) : 0;
+    if (part_bytes + order_bytes > 0) {
+        void* base = nullptr;
         if (fixed != nullptr) {
-            part = fixed->ptr;
+            base = fixed->ptr;
         } else {
             // host-side fault injection: the allocation fails as it would when the device
             // is out of memory (nothing is launched)
             if (std::getenv("GQA_FAULT_INJECT_ALLOC") != nullptr) return GQA_ERR_ALLOC;
             cudaMemPool_t pool = workspace_pool(dev);
-            if (pool == nullptr || cudaMallocFromPoolAsync(&ws, bytes, pool, stream) != cudaSuccess) {
+            if (pool == nullptr ||
+                cudaMallocFromPoolAsync(&ws, part_bytes + order_bytes, pool, stream) != cudaSuccess) {
                 cudaGetLastError();
                 return GQA_ERR_ALLOC;
             }
-            part = ws;
+            base = ws;
         }
-        p.o_part = static_cast<float*>(part);
-        p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
+        if (pl.splits > 1) {
+            p.o_part = static_cast<float*>(base);
+            p.lse_part = p.o_part + (size_t)pl.splits * rows * d;
+        }
+        if (order_bytes > 0) p.unit_order = reinterpret_cast<int*>(static_cast<char*>(base) + part_bytes);
     }
     if (!encode_out(&p.tm_o, pl.splits > 1 ? (const void*)p.o_part : (const void*)out,
                     pl.splits > 1 ? pl.splits * B : B, Sq, Hq, d, pl.pack ? g : 1,
@@ -514,6 +527,15 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
 
     const int slots = info.sms * gqa::fwd_ctas_per_sm(d, pl.nt);
     const int grid = (int)(pl.units < slots ? pl.units : slots);
+    if (p.unit_order != nullptr) {
+        int* order = const_cast<int*>(p.unit_order);
+        gqa::FwdParams q = p;
+        q.unit_order = nullptr;
+        if (gqa::launch_unit_order(q, pl.nt, grid, order, order + pl.units, stream) != cudaSuccess) {
+            if (ws) cudaFreeAsync(ws, stream);
+            return GQA_ERR_CUDA;
+        }
+    }
     if (gqa::launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) {
         if (ws) cudaFreeAsync(ws, stream);
         return GQA_ERR_CUDA;

@@ -61,6 +61,10 @@ struct FwdParams {
     int page_shift;    // log2(page_size)
     int page_rows;     // rows of one TMA box: min(page_size, 128)
     int num_pages;     // pages in the pool (a page coordinate past it reads zeros)
+    // Work order (NULL: position u is unit u).  With per-sequence lengths the units' work
+    // varies; a pre-pass on the device writes here, for every position u of the static
+    // stride, the unit to take there: heaviest first, dealt round by round over the CTAs.
+    const int* unit_order;
 };
 
 struct CombineParams {

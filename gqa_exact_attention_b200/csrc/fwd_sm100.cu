@@ -114,6 +114,7 @@ struct UnitGeom {
 template <int NT>
 __device__ __forceinline__ UnitGeom<NT> unit_geom(int u, const FwdParams& p) {
     // all divisions by run-time sizes are multiply-shift (FastDiv), computed on the host
+    if (p.unit_order != nullptr) u = __ldg(p.unit_order + u);
     UnitGeom<NT> g;
     uint32_t w, r, q, rem;
     fastdivmod((uint32_t)u, p.div_window, w, r);
@@ -1042,6 +1043,51 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
     }
 }
 
+// ---------------------------------------------------------------- unit order by work
+// With per-sequence key lengths the units' work varies from nothing to the capacity; a
+// static stride over them leaves the CTA that draws long sequences last.  This pre-pass
+// (one CTA) sorts the units by their key-block count, heaviest first (a counting sort;
+// counts above kBuckets - 1 share the top bucket), and deals them in rounds of `grid`
+// positions, alternating direction (round r gives its k-th heaviest unit to CTA k when r is
+// even, to CTA grid-1-k when r is odd; a last partial round goes in order).  order[u] is
+// the unit that position u of the kernel's static stride takes.  sorted_tmp holds n_units
+// entries.  The order only moves work between CTAs: every unit is still computed once.
+template <int NT>
+__global__ void __launch_bounds__(1024) gqa_unit_order_kernel(const __grid_constant__ FwdParams p,
+                                                              int grid, int* order,
+                                                              int* sorted_tmp) {
+    constexpr int kBuckets = 2048;
+    __shared__ int cnt[kBuckets];
+    for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    FwdParams q = p;
+    q.unit_order = nullptr;
+    auto bucket_of = [&](int u) {
+        const int n = unit_geom<NT>(u, q).nblk;
+        return kBuckets - 1 - (n < kBuckets - 1 ? n : kBuckets - 1);  // heaviest first
+    };
+    for (int u = threadIdx.x; u < p.n_units; u += blockDim.x) atomicAdd(&cnt[bucket_of(u)], 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {  // exclusive prefix sum (2048 entries, once)
+        int acc = 0;
+        for (int i = 0; i < kBuckets; ++i) {
+            const int c = cnt[i];
+            cnt[i] = acc;
+            acc += c;
+        }
+    }
+    __syncthreads();
+    for (int u = threadIdx.x; u < p.n_units; u += blockDim.x)
+        sorted_tmp[atomicAdd(&cnt[bucket_of(u)], 1)] = u;
+    __syncthreads();
+    const int full_rounds = p.n_units / grid;
+    for (int pos = threadIdx.x; pos < p.n_units; pos += blockDim.x) {
+        const int r = pos / grid, k = pos - r * grid;
+        const int src = (r < full_rounds && (r & 1)) ? r * grid + (grid - 1 - k) : pos;
+        order[pos] = sorted_tmp[src];
+    }
+}
+
 // ---------------------------------------------------------------- split-KV combine
 // One warp per output row (b, h, i): M = max_s lse_s, w_s = exp(lse_s - M),
 // lse = M + ln sum w_s, O = sum_s w_s O_s / sum_s w_s.
@@ -1151,6 +1197,15 @@ int fwd_ctas_per_sm(int hd, int nt) {
 cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, int grid, cudaStream_t stream) {
     if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2>(p, grid, stream) : launch_fwd_t<128, 1>(p, grid, stream);
     return nt == 2 ? launch_fwd_t<64, 2>(p, grid, stream) : launch_fwd_t<64, 1>(p, grid, stream);
+}
+
+cudaError_t launch_unit_order(const FwdParams& p, int nt, int grid, int* order, int* tmp,
+                              cudaStream_t stream) {
+    if (nt == 2)
+        gqa_unit_order_kernel<2><<<1, 1024, 0, stream>>>(p, grid, order, tmp);
+    else
+        gqa_unit_order_kernel<1><<<1, 1024, 0, stream>>>(p, grid, order, tmp);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const CombineParams& p, int hd, int num_sms, cudaStream_t stream) {

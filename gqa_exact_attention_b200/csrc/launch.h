@@ -12,6 +12,11 @@ namespace gqa {
 int fwd_ctas_per_sm(int hd, int nt);
 cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, int grid, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int hd, int num_sms, cudaStream_t stream);
+// Work order for the forward kernel launched with `grid` CTAs (p.unit_order is ignored):
+// order[u] for every u < p.n_units, heaviest units first, dealt over the CTAs; tmp holds
+// p.n_units ints.
+cudaError_t launch_unit_order(const FwdParams& p, int nt, int grid, int* order, int* tmp,
+                              cudaStream_t stream);
 // Device address of the library's status word on the current device (NULL on error).
 unsigned int* device_status_symbol();
 // The forward with its split-KV partials in caller-side fixed scratch of scratch_bytes

@@ -171,9 +171,13 @@ typedef enum { GQA_OUT_F32 = 0, GQA_OUT_BF16 = 1 } gqa_out_dtype;
  * Errors as gqa_attn_fwd, plus GQA_ERR_ALIGN for a cache_seqlens pointer that is not
  * 4-byte aligned.  Split-KV partials stay fp32 (allocated as for gqa_attn_fwd).  With
  * cache_seqlens given and num_splits = 0, the split count follows a rule for ragged
- * lengths (about three units per CTA slot, never fewer splits than the dense rule), so
- * the partials can exceed what gqa_attn_workspace_bytes reports for the same shape; at
- * most 16 splits of B * Hq * Sq * (d + 1) fp32 values.
+ * lengths (about three work units per CTA slot), so the partials can differ from what
+ * gqa_attn_workspace_bytes reports for the same shape; at most 16 splits of
+ * B * Hq * Sq * (d + 1) fp32 values.  With cache_seqlens given and a short query axis
+ * (one 128-row tile of rows per (sequence, head or group): decode), a small pre-pass on
+ * the device orders the work units by their key count, longest first, and deals them over
+ * the CTAs; its scratch is 8 bytes per work unit, taken with the partials from the same
+ * pool.  The order changes which CTA computes a unit, never the result.
  */
 GQA_API gqa_status gqa_attn_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache,
                                         const int* cache_seqlens, void* out, int out_dtype,
