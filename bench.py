@@ -15,9 +15,10 @@ headline (the step timed over --steps launches), the line carries:
 
 --impl reference times the fp64 CPU oracle (the only reference this project has) on the
 box's host cores, on bounded samples of the same workload.  Other flags (--B, --Sq, ...)
-select another shape for ad-hoc measurement; ``--sweep prefill|decode|kvcache|paged`` prints
+select another shape for ad-hoc measurement; ``--sweep prefill|decode|kvcache|paged|fp8`` prints
 one line per configuration of the batch-sensitivity sweep, the decode grid, the KV-cache
-entry point (per-sequence lengths, bf16 output), or the paged KV cache next to the dense one.
+entry point (per-sequence lengths, bf16 output), the paged KV cache next to the dense one, or
+the e4m3 entry point next to bf16 inputs of the same shapes.
 """
 from __future__ import annotations
 
@@ -582,6 +583,8 @@ def run_sweep(args):
         return run_sweep_kvcache(args, peaks)
     if args.sweep == "paged":
         return run_sweep_paged(args, peaks)
+    if args.sweep == "fp8":
+        return run_sweep_fp8(args, peaks)
     if args.sweep == "prefill":
         cases = [(B, 2048, 2048, c, pk, sp) for B in (16, 32, 64, 128, 256) for c in (1, 0)
                  for (pk, sp) in [(-1, 0), (0, 1), (1, 1), (0, 2), (1, 2), (0, 4), (1, 4)]]
@@ -752,6 +755,73 @@ def run_sweep_paged(args, peaks):
             torch.cuda.empty_cache()
 
 
+def run_sweep_fp8(args, peaks):
+    """Kernel-only timings of gqa_attn_fwd_fp8 (e4m3 Q, K, V with per-tensor scales, fp32
+    output) next to gqa_attn_fwd on bf16 inputs of the same shape, both under the automatic
+    schedule: the decode grid (Sk 2K/8K/32K, B 32/128/256) against the measured copy
+    bandwidth, and the prefill shape (B=64, Sq=Sk=2048, causal and not) against the e4m3
+    tensor rate taken as twice the measured bf16 rate (the nominal dense ratio).  Bytes
+    count 1 byte per Q/K/V element for e4m3, 2 for bf16."""
+    import torch
+
+    import gqa_exact_attention_b200 as G
+    import inputs
+    stream = torch.cuda.current_stream()
+    Hq, Hk, d = 32, 8, 128
+    scales = (1 / 16, 1 / 16, 1 / 8)
+    cases = [(B, 1, Sk, 0) for Sk in (2048, 8192, 32768) for B in (32, 128, 256)]
+    cases += [(64, 2048, 2048, c) for c in (1, 0)]
+
+    def timed(step):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if G.gqa_attn_device_status(reset=True) != 0:
+            raise SystemExit("an in-kernel bounded wait timed out")
+        return e0.elapsed_time(e1) / args.steps
+
+    for (B, Sq, Sk, causal) in cases:
+        out = torch.empty((B, Sq, Hq, d), dtype=torch.float32, device="cuda")
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
+        q = inputs.device_tensor(1001, inputs.TID_Q, (B, Sq, Hq, d))
+        k = inputs.device_tensor(1001, inputs.TID_K, (B, Sk, Hk, d))
+        v = inputs.device_tensor(1001, inputs.TID_V, (B, Sk, Hk, d))
+        ms_bf16 = timed(lambda: G.gqa_attn_fwd(q, k, v, out=out, lse=lse, causal=causal,
+                                               stream=stream))
+        del q, k, v
+        torch.cuda.empty_cache()
+        q = inputs.e4m3_device_tensor(1001, inputs.TID_Q, (B, Sq, Hq, d), scales[0])
+        k = inputs.e4m3_device_tensor(1001, inputs.TID_K, (B, Sk, Hk, d), scales[1])
+        v = inputs.e4m3_device_tensor(1001, inputs.TID_V, (B, Sk, Hk, d), scales[2])
+        ms = timed(lambda: G.gqa_attn_fwd_fp8(q, k, v, *scales, out=out, lse=lse, causal=causal,
+                                              stream=stream))
+        del q, k, v
+        torch.cuda.empty_cache()
+        fl = flops(B, Sq, Sk, Hq, d, causal)
+        io = 4 * B * Sq * Hq * d + 4 * B * Hq * Sq  # fp32 out + LSE
+        by8 = B * Sq * Hq * d + 2 * B * Sk * Hk * d + io
+        by16 = 2 * (B * Sq * Hq * d + 2 * B * Sk * Hk * d) + io
+        line = {"sweep": "fp8", "B": B, "Sq": Sq, "Sk": Sk, "causal": bool(causal),
+                "ms": round(ms, 4), "bf16_ms": round(ms_bf16, 4),
+                "speedup_over_bf16": round(ms_bf16 / ms, 3),
+                "tflops": round(fl / ms / 1e9, 1), "hbm_gbs": round(by8 / ms / 1e6, 1),
+                "bf16_hbm_gbs": round(by16 / ms_bf16 / 1e6, 1)}
+        if Sq > 1:
+            line["frac_of_e4m3_peak"] = round(fl / ms / 1e9 / (2 * peaks["bf16_tflops"]), 3)
+            line["frac_of_measured_bf16"] = round(fl / ms / 1e9 / peaks["bf16_tflops"], 3)
+        else:
+            line["frac_of_measured_hbm"] = round(by8 / ms / 1e6 / peaks["hbm_gbs"], 3)
+        print(json.dumps(line), flush=True)
+        del out, lse
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -773,7 +843,7 @@ def main():
                     help="skip the >= 1 s timed region of the main step")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode workload of the default line")
-    ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache", "paged"], default=None,
+    ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache", "paged", "fp8"], default=None,
                     help="print one line per configuration of the batch sweep or decode grid")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -16,7 +16,7 @@ import os
 __all__ = [
     "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes", "gqa_attn_status_string",
     "gqa_attn_device_status", "gqa_attn_fwd_noalloc", "gqa_attn_fwd_kvcache",
-    "gqa_attn_fwd_paged", "GqaError", "lib_path", "load",
+    "gqa_attn_fwd_paged", "gqa_attn_fwd_fp8", "GqaError", "lib_path", "load",
     "GQA_NOALLOC_SCRATCH_BYTES",
 ]
 
@@ -77,6 +77,8 @@ def load():
     L.gqa_attn_fwd_kvcache.restype = i
     L.gqa_attn_fwd_paged.argtypes = [p, p, p, p, i, p, i, i, p, i, p, i, i, i, i, i, f, i, i, i, p]
     L.gqa_attn_fwd_paged.restype = i
+    L.gqa_attn_fwd_fp8.argtypes = [p, p, p, f, f, f, p, p, i, p, i, i, i, i, i, i, f, i, i, i, p]
+    L.gqa_attn_fwd_fp8.restype = i
     _lib = L
     return L
 
@@ -263,5 +265,53 @@ def gqa_attn_fwd_paged(q, k_pages, v_pages, block_table, cache_seqlens, out=None
             q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
             int(block_table.shape[1]), cache_seqlens.data_ptr(), num_pages, page_size,
             out.data_ptr(), code, lse.data_ptr(), B, Sq, Hq, Hk, d, float(scale),
+            int(bool(causal)), int(pack_gqa), int(num_splits), stream.cuda_stream))
+    return out, lse
+
+
+def gqa_attn_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, cache_seqlens=None, out=None,
+                     lse=None, out_dtype=None, scale=None, causal=False, pack_gqa=-1,
+                     num_splits=0, stream=None):
+    """out, lse = gqa_attn_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, ...).
+
+    q [B, Sq, Hq, d], k and v [B, Sk, Hk, d]: e4m3 tensors (torch.float8_e4m3fn or the raw
+    bytes as torch.uint8); the values they stand for are q * q_scale, k * k_scale and
+    v * v_scale (per-tensor fp32 scales).  cache_seqlens as in gqa_attn_fwd_kvcache.  out is
+    fp32 or bf16 [B, Sq, Hq, d]; lse fp32 [B, Hq, Sq].  scale defaults to 1/sqrt(d).
+    """
+    import torch
+
+    B, Sq, Hq, d = q.shape
+    Sk, Hk = k.shape[1], k.shape[2]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.element_size() != 1 or not t.is_cuda or not t.is_contiguous() or \
+                t.dtype not in (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8)):
+            raise ValueError(f"{name} must be a contiguous e4m3 (or uint8) CUDA tensor")
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Sk, Hk, d] matching q")
+    if cache_seqlens is not None:
+        if (cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_contiguous()
+                or cache_seqlens.device != q.device or tuple(cache_seqlens.shape) != (B,)):
+            raise ValueError("cache_seqlens must be a contiguous int32 tensor [B] on q's device")
+    if out is None:
+        dt = torch.float32 if out_dtype is None else out_dtype
+        out = torch.empty((B, Sq, Hq, d), dtype=dt, device=q.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or not out.is_contiguous() \
+            or out.device != q.device or tuple(out.shape) != (B, Sq, Hq, d):
+        raise ValueError("out must be a contiguous fp32 or bf16 tensor [B, Sq, Hq, d] on q's device")
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError("lse must be a contiguous fp32 tensor [B, Hq, Sq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    code = GQA_OUT_BF16 if out.dtype == torch.bfloat16 else GQA_OUT_F32
+    with torch.cuda.device(q.device):
+        _check(load().gqa_attn_fwd_fp8(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
+            float(v_scale), None if cache_seqlens is None else cache_seqlens.data_ptr(),
+            out.data_ptr(), code, lse.data_ptr(), B, Sq, Sk, Hq, Hk, d, float(scale),
             int(bool(causal)), int(pack_gqa), int(num_splits), stream.cuda_stream))
     return out, lse

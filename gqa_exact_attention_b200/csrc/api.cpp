@@ -226,20 +226,24 @@ EncodeTiled get_encode_tiled() {
     return fn;
 }
 
-// bf16 tensor [B, S, H, d] as a 4-D map (d, H, S, B), 128-byte swizzle, zero fill out of
-// bounds, box (64, box_h, box_s, 1).
+// Tensor [B, S, H, d] as a 4-D map (d, H, S, B), zero fill out of bounds.  bf16: box
+// (64, box_h, box_s, 1), 128-byte swizzle (a box row is 128 bytes).  e4m3 (f8): box
+// (d, box_h, box_s, 1), one byte per element, 128-byte swizzle for d = 128 and 64-byte for
+// d = 64 (a box row is d bytes).
 bool encode_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int d, int box_h,
-                 int box_s) {
+                 int box_s, bool f8 = false) {
     EncodeTiled enc = get_encode_tiled();
     if (!enc) return false;
+    const cuuint64_t es = f8 ? 1 : 2;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)S * H * d * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
+    cuuint64_t strides[3] = {(cuuint64_t)d * es, (cuuint64_t)H * d * es, (cuuint64_t)S * H * d * es};
+    cuuint32_t box[4] = {f8 ? (cuuint32_t)d : 64u, (cuuint32_t)box_h, (cuuint32_t)box_s, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const CUtensorMapSwizzle sw =
+        (f8 && d == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    return enc(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+               const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // fp32 output [Bs, S, H, d] (Bs = B, or splits * B for the partials) as a 4-D map
@@ -381,6 +385,11 @@ size_t partial_bytes(int splits, int B, int Sq, int Hq, int d) {
     return (size_t)splits * (size_t)B * Hq * Sq * ((size_t)d + 1) * sizeof(float);
 }
 
+// e4m3 inputs: q, k, v hold one byte per element; the values are q8 * q_scale etc.
+struct Fp8 {
+    float q_scale = 1.f, k_scale = 1.f, v_scale = 1.f;
+};
+
 // A paged KV cache: k and v are page pools [num_pages, page_size, Hk, d]; key j of
 // sequence b is row j % page_size of page block_table[b * table_stride + j / page_size].
 struct Paged {
@@ -398,7 +407,8 @@ bool is_pow2(long long x) { return x > 0 && (x & (x - 1)) == 0; }
 gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seqlens_k, void* out,
                     bool out_bf16, float* lse, int B, int Sq, int Sk, int Hq, int Hk, int d,
                     float scale, int causal, int pack_gqa, int num_splits, void* stream_ptr,
-                    const Scratch* fixed = nullptr, const Paged* paged = nullptr) {
+                    const Scratch* fixed = nullptr, const Paged* paged = nullptr,
+                    const Fp8* f8 = nullptr) {
     if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
     // a paged cache's logical capacity is not a dense tensor: its pool is checked below
     gqa_status st = validate_shape(B, Sq, paged ? 1 : Sk, Hq, Hk, d, pack_gqa, num_splits);
@@ -439,17 +449,18 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     const int g = Hq / Hk;
 
     gqa::FwdParams p{};
-    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM))
+    const bool is_f8 = f8 != nullptr;
+    if (!encode_bshd(&p.tm_q, q, B, Sq, Hq, d, pl.pack ? g : 1, pl.pack ? pl.pos_per_tile : kBlockM, is_f8))
         return GQA_ERR_CUDA;
     if (paged == nullptr) {
-        if (!encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN) ||
-            !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN))
+        if (!encode_bshd(&p.tm_k, k, B, Sk, Hk, d, 1, kBlockN, is_f8) ||
+            !encode_bshd(&p.tm_v, v, B, Sk, Hk, d, 1, kBlockN, is_f8))
             return GQA_ERR_CUDA;
     } else {
         // the page pools as (d, Hk, page_size, num_pages), boxes of up to 128 rows
         const int rows = paged->page_size < kBlockN ? paged->page_size : kBlockN;
-        if (!encode_bshd(&p.tm_k, k, paged->num_pages, paged->page_size, Hk, d, 1, rows) ||
-            !encode_bshd(&p.tm_v, v, paged->num_pages, paged->page_size, Hk, d, 1, rows))
+        if (!encode_bshd(&p.tm_k, k, paged->num_pages, paged->page_size, Hk, d, 1, rows, is_f8) ||
+            !encode_bshd(&p.tm_v, v, paged->num_pages, paged->page_size, Hk, d, 1, rows, is_f8))
             return GQA_ERR_CUDA;
         p.block_table = paged->block_table;
         p.table_stride = paged->table_stride;
@@ -480,7 +491,10 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     p.batch_window = batch_window(B, Sk, Hk, d);
     set_unit_divisors(&p, B);
     p.kv_blocks = pl.kv_blocks;
-    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    // e4m3: the scores are q8 . k8 * q_scale * k_scale, and O carries v_scale
+    const double qk = is_f8 ? (double)f8->q_scale * (double)f8->k_scale : 1.0;
+    p.scale_log2 = (float)((double)scale * qk * 1.4426950408889634);
+    p.v_scale = is_f8 ? f8->v_scale : 1.f;
     p.div_g = gqa::make_fastdiv((uint32_t)g);
     p.status = nullptr;
     p.timeout_ns = timeout_ns();
@@ -536,7 +550,7 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
             return GQA_ERR_CUDA;
         }
     }
-    if (gqa::launch_fwd(p, d, pl.nt, grid, stream) != cudaSuccess) {
+    if (gqa::launch_fwd(p, d, pl.nt, is_f8, grid, stream) != cudaSuccess) {
         if (ws) cudaFreeAsync(ws, stream);
         return GQA_ERR_CUDA;
     }
@@ -630,6 +644,23 @@ gqa_status gqa_attn_fwd_paged(const void* q, const void* k_pages, const void* v_
     return fwd_impl(q, k_pages, v_pages, cache_seqlens, out, out_dtype == GQA_OUT_BF16, lse, B,
                     Sq, max_pages_per_seq * page_size, Hq, Hk, d, scale, causal, pack_gqa,
                     num_splits, stream, nullptr, &pg);
+}
+
+gqa_status gqa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale,
+                            float k_scale, float v_scale, const int* cache_seqlens, void* out,
+                            int out_dtype, float* lse, int B, int Sq, int Sk, int Hq, int Hk,
+                            int d, float scale, int causal, int pack_gqa, int num_splits,
+                            void* stream) {
+    if (out_dtype != GQA_OUT_F32 && out_dtype != GQA_OUT_BF16) return GQA_ERR_SHAPE;
+    if (!std::isfinite(q_scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale) ||
+        !(q_scale > 0.f) || !(k_scale > 0.f) || !(v_scale > 0.f))
+        return GQA_ERR_SHAPE;
+    Fp8 f8;
+    f8.q_scale = q_scale;
+    f8.k_scale = k_scale;
+    f8.v_scale = v_scale;
+    return fwd_impl(q, k, v, cache_seqlens, out, out_dtype == GQA_OUT_BF16, lse, B, Sq, Sk, Hq, Hk,
+                    d, scale, causal, pack_gqa, num_splits, stream, nullptr, nullptr, &f8);
 }
 
 gqa_status gqa_attn_device_status(int reset) {

@@ -65,6 +65,9 @@ struct FwdParams {
     // varies; a pre-pass on the device writes here, for every position u of the static
     // stride, the unit to take there: heaviest first, dealt round by round over the CTAs.
     const int* unit_order;
+    // e4m3 inputs: V's per-tensor scale, applied to O in the epilogue (1 for bf16 inputs;
+    // Q's and K's scales are folded into scale_log2)
+    float v_scale;
 };
 
 struct CombineParams {

@@ -41,12 +41,27 @@ namespace {
 
 using namespace ptx;
 
-template <int HD, int NT>
+// F8: Q, K, V in e4m3 (one byte per element), MMAs of kind::f8f6f4, P in e4m3.
+template <int HD, int NT, bool F8 = false>
 struct FwdCfg {
-    static constexpr int kChunks = HD / 64;              // 128-byte column chunks of a row
-    static constexpr int kChunkBytes = 128 * 128;        // 128 rows x 128 bytes
+    static constexpr int kRowBytes = F8 ? HD : 2 * HD;   // one row of Q, K or V
+    // a tile is kChunks column chunks of 128 rows; a chunk row is at most 128 bytes (the
+    // swizzle span): bf16 rows split into 64-column chunks, e4m3 rows (64 or 128 bytes) fit
+    static constexpr int kChunks = F8 ? 1 : HD / 64;
+    static constexpr int kChunkRowBytes = F8 ? kRowBytes : 128;
+    static constexpr int kChunkBytes = 128 * kChunkRowBytes;
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kSlots = (NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 2 : 5);
+    static constexpr int kSlots = (F8 ? 2 : 1) * ((NT == 2) ? (HD == 128 ? 4 : 8) : (HD == 128 ? 2 : 5));
+    // shared-memory operand layout: 128-byte swizzle (atoms of 8 rows x 128 bytes), or
+    // 64-byte swizzle for 64-byte rows
+    static constexpr bool kSw64 = kChunkRowBytes == 64;
+    static constexpr uint32_t kAtomBytes = 8 * kChunkRowBytes;
+    // MMA K per instruction (16 bf16 or 32 e4m3 = 32 bytes) and steps per 128-key P.V
+    static constexpr int kMmaK = F8 ? 32 : 16;
+    static constexpr int kPvSteps = kBlockN / kMmaK;
+    static constexpr uint32_t kPvStepBytes = kMmaK * kChunkRowBytes;  // keys of one step, one chunk
+    // TMEM columns of P per 32-key chunk (2 bf16 or 4 e4m3 per column)
+    static constexpr int kPColsPer32 = F8 ? 8 : 16;
     // NT == 2: warpgroups 0 = TMA producer + MMA issuer, 1..2 = softmax (one per tile),
     //          3 = epilogue; one CTA per SM.
     // NT == 1: warpgroup 0 as above, 1 = softmax that also writes its tile's output; two
@@ -80,8 +95,19 @@ struct FwdCfg {
                                       kSlots * kTileBytes + kOStageBytes + 8 * kNumBars +
                                       kStatsBytes + 16;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-    static constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);
-    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, HD, true);
+    static constexpr uint32_t kIdescQK = F8 ? idesc_e4m3_f32(128, 128, false) : idesc_bf16_f32(128, 128, false);
+    static constexpr uint32_t kIdescPV = F8 ? idesc_e4m3_f32(128, HD, true) : idesc_bf16_f32(128, HD, true);
+    __device__ static uint64_t sdesc(uint32_t saddr, uint32_t lbo) {
+        return kSw64 ? sdesc_sw64(saddr, lbo, kAtomBytes) : sdesc_sw128(saddr, lbo, kAtomBytes);
+    }
+    __device__ static void mma_s(uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
+        if constexpr (F8) mma_ss_f8(d, a, b, kIdescQK, acc);
+        else mma_ss(d, a, b, kIdescQK, acc);
+    }
+    __device__ static void mma_pv(uint32_t d, uint32_t a, uint64_t b, uint32_t acc) {
+        if constexpr (F8) mma_ts_f8(d, a, b, kIdescPV, acc);
+        else mma_ts(d, a, b, kIdescPV, acc);
+    }
     __host__ __device__ static constexpr int s_col(int t) { return t * 128; }
     __host__ __device__ static constexpr int o_col(int t) { return NT * 128 + t * HD; }
 };
@@ -194,7 +220,7 @@ __device__ __forceinline__ void write_row(const FwdParams& p, uint32_t o_addr, c
                                           int b, int split, bool has, bool idle, float m, float l,
                                           uint32_t o_empty_bar) {
     constexpr float kLn2 = 0.69314718055994530942f;
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    const float inv_l = (l > 0.f) ? p.v_scale / l : 0.f;
     const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
     float* orow = nullptr;
     float* lrow;
@@ -323,10 +349,10 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const 
     }
 }
 
-template <int HD, int NT>
-__global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCtasPerSm)
+template <int HD, int NT, bool F8>
+__global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F8>::kCtasPerSm)
     gqa_fwd_kernel(const __grid_constant__ FwdParams p) {
-    using C = FwdCfg<HD, NT>;
+    using C = FwdCfg<HD, NT, F8>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -412,7 +438,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 if (!ok) return;
                 if (elect_one()) {
                     const int rows = p.pack ? p.rows_valid : kBlockM;
-                    mbar_arrive_expect_tx(q_full(t), (uint32_t)(C::kChunks * rows * 128));
+                    mbar_arrive_expect_tx(q_full(t), (uint32_t)(rows * C::kRowBytes));
                     const int hcoord = p.pack ? g.hg * p.g : g.hg;
 #pragma unroll
                     for (int c = 0; c < C::kChunks; ++c)
@@ -467,7 +493,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
 #pragma unroll
                                     for (int c = 0; c < C::kChunks; ++c)
                                         tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes +
-                                                        sub * p.page_rows * 128,
+                                                        sub * p.page_rows * C::kChunkRowBytes,
                                                     tm, kv_full(slot), c * 64, g.kvh, prow[sub], pg[sub]);
                                 }
                             }
@@ -498,9 +524,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
             uint32_t qn[NT] = {}, pn[NT] = {}, on[NT] = {};
             bool ok = true;
             // descriptors built once; each MMA advances them by a constant offset
-            const uint64_t q_desc0 = sdesc_sw128(sQ, 16, 1024);
-            const uint64_t k_desc0 = sdesc_sw128(sKV, 16, 1024);
-            const uint64_t v_desc0 = sdesc_sw128(sKV, C::kChunkBytes, 1024);
+            const uint64_t q_desc0 = C::sdesc(sQ, 16);
+            const uint64_t k_desc0 = C::sdesc(sKV, 16);
+            const uint64_t v_desc0 = C::sdesc(sKV, C::kChunkBytes);  // MN-major: chunks along d
             // Issue a group of MMAs; before its last MMA, probe (without blocking) the
             // barrier the next group will wait on, so the probe's latency overlaps that
             // MMA instead of leaving the tensor pipe idle.  Returns the probe's result.
@@ -510,12 +536,13 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 const uint32_t d = tmem + C::s_col(t);
                 bool ready = false;
                 if (elect_one()) {
+                    // 32 bytes of the row per MMA: 16 bf16 or 32 e4m3 of d
+                    constexpr int kSteps = C::kRowBytes / 32;
 #pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
+                    for (int kk = 0; kk < kSteps; ++kk) {
                         const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                        if (kk == HD / 16 - 1 && probe_bar != 0u) ready = mbar_test_wait(probe_bar, probe_par);
-                        mma_ss(d, sdesc_add(a0, off), sdesc_add(b0, off), C::kIdescQK,
-                               kk > 0 ? 1u : 0u);
+                        if (kk == kSteps - 1 && probe_bar != 0u) ready = mbar_test_wait(probe_bar, probe_par);
+                        C::mma_s(d, sdesc_add(a0, off), sdesc_add(b0, off), kk > 0 ? 1u : 0u);
                     }
                 }
                 return __ballot_sync(0xffffffffu, ready) != 0u;  // only the issuing lane probed
@@ -528,11 +555,12 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 const uint32_t a = tmem + C::s_col(t);
                 bool ready = false;
                 if (elect_one()) {
+                    // 8 TMEM columns of P per MMA (16 bf16 or 32 e4m3 keys)
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                        if (kk == kBlockN / 16 - 1 && probe_bar != 0u) ready = mbar_test_wait(probe_bar, probe_par);
-                        mma_ts(d, a + kk * 8, sdesc_add(b0, kk * 2048), C::kIdescPV,
-                               (accumulate || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < C::kPvSteps; ++kk) {
+                        if (kk == C::kPvSteps - 1 && probe_bar != 0u) ready = mbar_test_wait(probe_bar, probe_par);
+                        C::mma_pv(d, a + kk * 8, sdesc_add(b0, kk * C::kPvStepBytes),
+                                  (accumulate || kk > 0) ? 1u : 0u);
                     }
                 }
                 return __ballot_sync(0xffffffffu, ready) != 0u;  // only the issuing lane probed
@@ -799,11 +827,18 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 // schedule, so x = c s is rounded once, the same way whether the key axis is
                 // split or the heads packed, and P is bit-identical across the scheduling
                 // variants; where m does move, it moves by integers, so p changes by exact
-                // powers of two and the rescale factors are exact.
-                const bool grow = mx > m + 8.0f || (l == 0.f && mx > kNegInf && mx < m - 64.f);
+                // powers of two and the rescale factors are exact.  With e4m3 P, whose
+                // smallest value is 2^-9 and whose normals start at 2^-6, the lower edge is
+                // m - 1 and a move leaves the block max 4 octaves above m (p_max in (8, 16]):
+                // the row's largest p is then always >= 1/2 (m <= the row max + 1), and keys
+                // up to 9 octaves below the max keep e4m3's full 3-bit precision.  Moves are
+                // still by integers, and e4m3 rounding commutes with powers of two.
+                constexpr float kLowEdge = F8 ? 1.0f : 64.f;
+                constexpr float kHeadroom = F8 ? 4.0f : 0.f;
+                const bool grow = mx > m + 8.0f || (l == 0.f && mx > kNegInf && mx < m - kLowEdge);
                 float alpha = 1.f;
                 if (grow) {
-                    const float m_new = ceilf(mx);
+                    const float m_new = ceilf(mx) - kHeadroom;
                     alpha = (l == 0.f) ? 0.f : ex2_approx(m - m_new);  // nothing summed: O is 0
                     l *= alpha;
                     m = m_new;
@@ -814,11 +849,24 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 float ls0 = 0.f, ls1 = 0.f;
                 // the pairs of a chunk that take the polynomial, spread over the chunk
                 auto use_poly = [](int ch, int i) { return ((i * 5 + ch * 3) & 15) < C::kPolyPairs; };
+                // P of 32-key chunk ch into TMEM over S: 16 columns of bf16 pairs, or 8 of e4m3
+                // quads (pk[0..7])
+                auto store_p = [&](int ch, const uint32_t (&pk)[16]) {
+                    if constexpr (F8) {
+                        uint32_t q8[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) q8[i] = pk[i];
+                        tmem_st8(s_addr + ch * C::kPColsPer32, q8);
+                    } else {
+                        tmem_st16(s_addr + ch * C::kPColsPer32, pk);
+                    }
+                };
                 // one 32-key chunk: P = 2^(c s - m) as bf16 pairs; with kSelect, keys at or
                 // past lim get the exponent -inf (p = 0 for either sign of c)
                 auto exp_chunk = [&](auto select_c, int ch) {
                     constexpr bool kSelect = decltype(select_c)::value;
-                    uint32_t pk[16];
+                    uint32_t pk[16];  // P of the chunk: 16 bf16 pairs, or 8 e4m3 quads
+                    [[maybe_unused]] float p_even0 = 0.f, p_even1 = 0.f;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int j = ch * 32 + 2 * i;
@@ -836,9 +884,17 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                             p1 = ex2_approx(x1);
                         }
                         add2(ls0, ls1, p0, p1, ls0, ls1);
-                        pk[i] = pack_bf16x2(p0, p1);
+                        if constexpr (F8) {
+                            if (i & 1) pk[i >> 1] = pack_e4m3x4(p_even0, p_even1, p0, p1);
+                            else {
+                                p_even0 = p0;
+                                p_even1 = p1;
+                            }
+                        } else {
+                            pk[i] = pack_bf16x2(p0, p1);
+                        }
                     }
-                    tmem_st16(s_addr + ch * 16, pk);
+                    store_p(ch, pk);
                 };
                 auto exp_range = [&](auto masked_c, int ch0, int ch1) {
                     constexpr bool kMasked = decltype(masked_c)::value;
@@ -849,8 +905,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                         } else if (chunk_empty(ch)) {
                             uint32_t pk[16];
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) pk[i] = 0u;  // two bf16 zeros
-                            tmem_st16(s_addr + ch * 16, pk);
+                            for (int i = 0; i < 16; ++i) pk[i] = 0u;  // zeros in either format
+                            store_p(ch, pk);
                         } else {
                             exp_chunk(std::true_type{}, ch);
                         }
@@ -936,7 +992,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT>::kThreads, FwdCfg<HD, NT>::kCta
                 ok = named_bar_and(kEpiBar, 128, ok);
                 if (!ok) break;
                 tc_fence_after();
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                const float inv_l = (l > 0.f) ? p.v_scale / l : 0.f;
                 const float lse_v = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
                 const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
                 const int hcoord = p.pack ? g.hg * p.g : g.hg;
@@ -1159,15 +1215,15 @@ __global__ void __launch_bounds__(256) gqa_combine_kernel(const CombineParams p)
     }
 }
 
-template <int HD, int NT>
+template <int HD, int NT, bool F8>
 cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
-    using C = FwdCfg<HD, NT>;
+    using C = FwdCfg<HD, NT, F8>;
     // the attribute is per device; setting it again is idempotent, so the race is benign
     static bool configured[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_fwd_kernel<HD, NT>,
+        cudaError_t e = cudaFuncSetAttribute(gqa_fwd_kernel<HD, NT, F8>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
@@ -1178,12 +1234,12 @@ cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
     static int regs_checked = 0;  // 0 unknown, 1 ok, -1 mismatch
     if (regs_checked == 0) {
         cudaFuncAttributes attr{};
-        cudaError_t e = cudaFuncGetAttributes(&attr, gqa_fwd_kernel<HD, NT>);
+        cudaError_t e = cudaFuncGetAttributes(&attr, gqa_fwd_kernel<HD, NT, F8>);
         if (e != cudaSuccess) return e;
         regs_checked = (attr.numRegs == C::kLaunchRegs) ? 1 : -1;
     }
     if (regs_checked != 1) return cudaErrorInvalidConfiguration;
-    gqa_fwd_kernel<HD, NT><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+    gqa_fwd_kernel<HD, NT, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -1194,9 +1250,13 @@ int fwd_ctas_per_sm(int hd, int nt) {
     return hd == 128 ? FwdCfg<128, 1>::kCtasPerSm : FwdCfg<64, 1>::kCtasPerSm;
 }
 
-cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, int grid, cudaStream_t stream) {
-    if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2>(p, grid, stream) : launch_fwd_t<128, 1>(p, grid, stream);
-    return nt == 2 ? launch_fwd_t<64, 2>(p, grid, stream) : launch_fwd_t<64, 1>(p, grid, stream);
+cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, bool f8, int grid, cudaStream_t stream) {
+    if (f8) {
+        if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, true>(p, grid, stream) : launch_fwd_t<128, 1, true>(p, grid, stream);
+        return nt == 2 ? launch_fwd_t<64, 2, true>(p, grid, stream) : launch_fwd_t<64, 1, true>(p, grid, stream);
+    }
+    if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, false>(p, grid, stream) : launch_fwd_t<128, 1, false>(p, grid, stream);
+    return nt == 2 ? launch_fwd_t<64, 2, false>(p, grid, stream) : launch_fwd_t<64, 1, false>(p, grid, stream);
 }
 
 cudaError_t launch_unit_order(const FwdParams& p, int nt, int grid, int* order, int* tmp,

@@ -10,7 +10,8 @@ namespace gqa {
 
 // CTAs of the forward kernel resident per SM for (head dim, tiles per CTA).
 int fwd_ctas_per_sm(int hd, int nt);
-cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, int grid, cudaStream_t stream);
+// f8: e4m3 Q, K, V (kind::f8f6f4 MMAs); else bf16.
+cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, bool f8, int grid, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int hd, int num_sms, cudaStream_t stream);
 // Work order for the forward kernel launched with `grid` CTAs (p.unit_order is ignored):
 // order[u] for every u < p.n_units, heaviest units first, dealt over the CTAs; tmp holds

@@ -224,6 +224,38 @@ GQA_API gqa_status gqa_attn_fwd_paged(const void* q, const void* k_pages, const 
                                       int Hk, int d, float scale, int causal, int pack_gqa,
                                       int num_splits, void* stream);
 
+/*
+ * gqa_attn_fwd_fp8 — the forward of gqa_attn_fwd_kvcache with 8-bit inputs: Q, K and V
+ * in e4m3 (OCP FP8 E4M3: 4 exponent bits, bias 7, 3 mantissa bits, largest finite 448)
+ * with one fp32 scale per tensor.
+ *
+ * The pages recommend FP8 for the intermediate computation to halve the bandwidth
+ * pressure of attention ("解锁Stable Diffusion效率瓶颈…", "行业应用场景拓展", scenario two,
+ * "FP16输入，FP8中间计算"; "三步优化检查清单", step one; "為什么 GQA 推理吞吐先升后降…",
+ * "驗證與進階"; "PyTorch 性能分析深度指南 (第三部分)", "总结与建议", 混合精度).
+ *
+ *   q, k, v             e4m3 bytes, [B, Sq, Hq, d] and [B, Sk, Hk, d], 16-byte aligned.
+ *   q_scale, k_scale, v_scale   finite, > 0: the inputs stand for q * q_scale, k * k_scale
+ *                       and v * v_scale, and the result is the attention of those values.
+ *   cache_seqlens       NULL, or per-sequence key counts as in gqa_attn_fwd_kvcache.
+ *   other arguments     as gqa_attn_fwd_kvcache (fp32 or bf16 out, fp32 lse).
+ *
+ * How it computes: Q K^T in e4m3 with fp32 accumulation; the softmax in fp32 as for bf16
+ * inputs; P rounded to e4m3 (to nearest even) for P V, also with fp32 accumulation.  The
+ * row sums keep the unrounded P, and each row's largest p is at least 1/2.  Relative to the
+ * exact attention of the scaled inputs, an output element's error is then at most
+ * 2^-4 * sum_j w_j |v_j| + 2^-9 * max_j w_j * sum_j |v_j| (w_j the exact softmax weights)
+ * plus fp32 rounding; the LSE carries only fp32 rounding.
+ *
+ * Errors as gqa_attn_fwd_kvcache; GQA_ERR_SHAPE also for a scale that is not finite and
+ * positive.
+ */
+GQA_API gqa_status gqa_attn_fwd_fp8(const void* q, const void* k, const void* v, float q_scale,
+                                    float k_scale, float v_scale, const int* cache_seqlens,
+                                    void* out, int out_dtype, float* lse, int B, int Sq, int Sk,
+                                    int Hq, int Hk, int d, float scale, int causal, int pack_gqa,
+                                    int num_splits, void* stream);
+
 /* Static description of a status code. */
 GQA_API const char* gqa_attn_status_string(gqa_status status);
 

@@ -60,6 +60,10 @@ def _host_lib():
         lib.gqa_gen_bf16_range.restype = None
         lib.gqa_gen_bf16_strided.argtypes = [u64, u64, u64, u64, u64, u64, p]
         lib.gqa_gen_bf16_strided.restype = None
+        lib.gqa_e4m3_rne_from_double.argtypes = [ctypes.c_double]
+        lib.gqa_e4m3_rne_from_double.restype = ctypes.c_uint8
+        lib.gqa_gen_e4m3_range.argtypes = [u64, u64, u64, u64, ctypes.c_double, p]
+        lib.gqa_gen_e4m3_range.restype = None
         _host = lib
     return _host
 
@@ -72,6 +76,8 @@ def _dev_lib():
         u64, p = ctypes.c_uint64, ctypes.c_void_p
         lib.gqa_gen_bf16_device.argtypes = [u64, u64, u64, u64, p, p]
         lib.gqa_gen_bf16_device.restype = ctypes.c_int
+        lib.gqa_gen_e4m3_device.argtypes = [u64, u64, u64, u64, ctypes.c_double, p, p]
+        lib.gqa_gen_e4m3_device.restype = ctypes.c_int
         _dev = lib
     return _dev
 
@@ -128,6 +134,50 @@ def device_tensor(seed: int, tid: int, shape, device="cuda", stream=None):
     if n:
         s = stream if stream is not None else torch.cuda.current_stream(t.device)
         rc = _dev_lib().gqa_gen_bf16_device(seed, tid, 0, n, t.data_ptr(), s.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"device input generator failed (code {rc})")
+    return t
+
+
+# ------------------------------------------------------------------ e4m3 (8-bit) inputs
+
+def e4m3_bits_to_f64(bits: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """Exact value of e4m3 bit patterns (uint8) times scale, in float64 (0x7F/0xFF, the
+    format's NaN, never come out of the generator)."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 15
+    m = (b & 7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    return sign * mag * scale
+
+
+def e4m3_encode(t) -> np.ndarray:
+    """e4m3 bit patterns of the values t (round to nearest even, saturating), with the
+    generator's own encoder."""
+    lib = _host_lib()
+    flat = np.asarray(t, dtype=np.float64).ravel()
+    return np.array([lib.gqa_e4m3_rne_from_double(float(x)) for x in flat],
+                    dtype=np.uint8).reshape(np.shape(t))
+
+
+def e4m3_bits_tensor(seed: int, tid: int, shape, scale: float) -> np.ndarray:
+    """e4m3(z / scale) for the whole tensor, as uint8 bit patterns."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint8)
+    if n:
+        _host_lib().gqa_gen_e4m3_range(seed, tid, 0, n, float(scale), out.ctypes.data)
+    return out.reshape(shape)
+
+
+def e4m3_device_tensor(seed: int, tid: int, shape, scale: float, device="cuda", stream=None):
+    """The e4m3 tensor generated in device memory, as torch.uint8 (same bits as the host)."""
+    import torch
+    t = torch.empty(tuple(shape), dtype=torch.uint8, device=device)
+    n = t.numel()
+    if n:
+        s = stream if stream is not None else torch.cuda.current_stream(t.device)
+        rc = _dev_lib().gqa_gen_e4m3_device(seed, tid, 0, n, float(scale), t.data_ptr(), s.cuda_stream)
         if rc != 0:
             raise RuntimeError(f"device input generator failed (code {rc})")
     return t

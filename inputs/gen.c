@@ -61,3 +61,30 @@ void gqa_gen_bf16_strided(uint64_t seed, uint64_t tensor_id, uint64_t offset, ui
             out[(uint64_t)o * inner + n] = bf16_rne_from_double(
                 normal_from_counter(base, offset + (uint64_t)o * outer_stride + n));
 }
+
+uint8_t gqa_e4m3_rne_from_double(double t) {
+    const uint8_t sign = signbit(t) ? 0x80u : 0u;
+    const double a = fabs(t);
+    if (a == 0.0) return sign;
+    if (!(a < 448.0)) return (uint8_t)(sign | 0x7Eu); /* 448 and above (and NaN): +-448 */
+    int e = ilogb(a);                                   /* a in [2^e, 2^(e+1)) */
+    if (e < -6) {                                       /* subnormal: m * 2^-9, m in [0, 8] */
+        const double m = nearbyint(ldexp(a, 9));        /* exact scaling; ties to even */
+        return (uint8_t)(sign | (uint8_t)m);            /* m = 8 is the smallest normal */
+    }
+    double q = nearbyint(ldexp(a, 3 - e));              /* 4 significant bits: [8, 16] */
+    if (q == 16.0) {
+        q = 8.0;
+        ++e;
+    }
+    return (uint8_t)(sign | (uint8_t)(((e + 7) << 3) | ((int)q - 8)));
+}
+
+void gqa_gen_e4m3_range(uint64_t seed, uint64_t tensor_id, uint64_t start, uint64_t count,
+                        double scale, uint8_t* out) {
+    const uint64_t base = tensor_base(seed, tensor_id);
+    long long n = (long long)count;
+#pragma omp parallel for schedule(static)
+    for (long long t = 0; t < n; ++t)
+        out[t] = gqa_e4m3_rne_from_double(normal_from_counter(base, start + (uint64_t)t) / scale);
+}

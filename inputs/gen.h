@@ -23,6 +23,11 @@
  * rounding midpoint (probability ~2^-44 per element).
  *
  * Tensor ids used by the tests and the benchmark: Q = 1, K = 2, V = 3.
+ *
+ * e4m3 variant (for 8-bit inputs): element = e4m3(z / scale), where e4m3(t) rounds t to
+ * the OCP FP8 E4M3 format (4 exponent bits, bias 7, 3 mantissa bits, subnormals m * 2^-9,
+ * no infinities, largest finite 448) to nearest even, saturating at +-448; again exact
+ * integer/ldexp arithmetic from fp64.  The value it stands for is e4m3_value(bits) * scale.
  */
 #ifndef GQA_INPUTS_GEN_H
 #define GQA_INPUTS_GEN_H
@@ -44,6 +49,13 @@ void gqa_gen_bf16_range(uint64_t seed, uint64_t tensor_id, uint64_t start, uint6
  * n < inner, o < outer.  Used to regenerate one head's K/V rows of a BSHD tensor. */
 void gqa_gen_bf16_strided(uint64_t seed, uint64_t tensor_id, uint64_t offset, uint64_t inner,
                           uint64_t outer, uint64_t outer_stride, uint16_t* out);
+
+/* e4m3 bit pattern of t (round to nearest even, saturating at +-448). */
+uint8_t gqa_e4m3_rne_from_double(double t);
+
+/* out[n] = e4m3(z_(start + n) / scale), n < count.  Multithreaded (OpenMP). */
+void gqa_gen_e4m3_range(uint64_t seed, uint64_t tensor_id, uint64_t start, uint64_t count,
+                        double scale, uint8_t* out);
 
 #ifdef __cplusplus
 }

@@ -40,7 +40,63 @@ __global__ void gen_bf16_kernel(uint64_t base, uint64_t start, uint64_t count, u
     }
 }
 
+__device__ __forceinline__ uint8_t e4m3_rne_from_double(double t) {
+    const uint8_t sign = signbit(t) ? 0x80u : 0u;
+    const double a = fabs(t);
+    if (a == 0.0) return sign;
+    if (!(a < 448.0)) return (uint8_t)(sign | 0x7Eu);
+    int e = ilogb(a);
+    if (e < -6) return (uint8_t)(sign | (uint8_t)rint(ldexp(a, 9)));
+    double q = rint(ldexp(a, 3 - e));
+    if (q == 16.0) {
+        q = 8.0;
+        ++e;
+    }
+    return (uint8_t)(sign | (uint8_t)(((e + 7) << 3) | ((int)q - 8)));
+}
+
+__global__ void gen_e4m3_kernel(uint64_t base, uint64_t start, uint64_t count, double scale,
+                                uint8_t* out) {
+    uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t t = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; t < count; t += stride) {
+        uint64_t r = mix64(base + (start + t + 1) * kGolden);
+        double u1 = (double)((r >> 40) + 1) * (1.0 / 16777216.0);
+        double u2 = (double)((r >> 16) & 0xFFFFFFull) * (1.0 / 16777216.0);
+        double z = sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+        out[t] = e4m3_rne_from_double(z / scale);
+    }
+}
+
+uint64_t tensor_base(uint64_t seed, uint64_t tensor_id) {
+    uint64_t base = seed * kGolden + tensor_id;
+    base ^= base >> 30;
+    base *= 0xbf58476d1ce4e5b9ull;
+    base ^= base >> 27;
+    base *= 0x94d049bb133111ebull;
+    base ^= base >> 31;
+    return base;
+}
+
+unsigned grid_for(uint64_t count) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    uint64_t blocks = (count + 255) / 256;
+    uint64_t cap = (uint64_t)sms * 16;
+    return (unsigned)(blocks > cap ? cap : blocks);
+}
+
 }  // namespace
+
+extern "C" int gqa_gen_e4m3_device(uint64_t seed, uint64_t tensor_id, uint64_t start,
+                                   uint64_t count, double scale, uint8_t* out,
+                                   cudaStream_t stream) {
+    if (count == 0) return 0;
+    if (out == nullptr) return 1;
+    gen_e4m3_kernel<<<grid_for(count), 256, 0, stream>>>(tensor_base(seed, tensor_id), start,
+                                                         count, scale, out);
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
 
 extern "C" int gqa_gen_bf16_device(uint64_t seed, uint64_t tensor_id, uint64_t start,
                                    uint64_t count, uint16_t* out, cudaStream_t stream) {

@@ -22,7 +22,7 @@ def test_header_declares_the_entry_points():
     assert declared_symbols() == sorted([
         "gqa_attn_fwd", "gqa_attn_choose", "gqa_attn_workspace_bytes",
         "gqa_attn_status_string", "gqa_attn_device_status", "gqa_attn_fwd_noalloc",
-        "gqa_attn_fwd_kvcache", "gqa_attn_fwd_paged"])
+        "gqa_attn_fwd_kvcache", "gqa_attn_fwd_paged", "gqa_attn_fwd_fp8"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -112,6 +112,23 @@ def test_paged_invalid_arguments(kw, code):
     assert paged_raw(**kw) == code
 
 
+def fp8_raw(q=16, k=16, v=16, qs=1.0, ks=1.0, vs=1.0, seqlens=NULL, out=16, out_dtype=0, lse=16,
+            B=1, Sq=8, Sk=8, Hq=4, Hk=2, d=64, scale=0.125, causal=0, pack=-1, splits=0):
+    L = G.load()
+    return L.gqa_attn_fwd_fp8(q, k, v, qs, ks, vs, seqlens, out, out_dtype, lse, B, Sq, Sk, Hq,
+                              Hk, d, scale, causal, pack, splits, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qs=0.0), 2), (dict(ks=-1.0), 2), (dict(vs=float("inf")), 2), (dict(qs=float("nan")), 2),
+    (dict(out_dtype=3), 2), (dict(q=NULL), 1), (dict(v=NULL), 1), (dict(lse=NULL), 1),
+    (dict(q=24), 5), (dict(seqlens=18), 5), (dict(Hq=6, Hk=4), 3), (dict(d=96), 4), (dict(Sk=0), 2),
+])
+def test_fp8_invalid_arguments(kw, code):
+    # fake pointers: rejected on the host before anything is launched or read
+    assert fp8_raw(**kw) == code
+
+
 def test_pages_head_constraint_example():
     """Hq must be a multiple of Hk (the pages' interface constraint); Hq=6, Hk=2 is valid."""
     L = G.load()
@@ -175,3 +192,4 @@ def test_no_gpu_is_an_error_not_a_fallback():
     L = G.load()
     assert L.gqa_attn_fwd_noalloc(16, 16, 16, 16, 16, 1, 8, 8, 4, 2, 64, 0.125, 0, -1, 0, None) in (6, 8)
     assert paged_raw() in (6, 8)
+    assert fp8_raw() in (6, 8)
