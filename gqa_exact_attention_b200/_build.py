@@ -39,7 +39,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cmd = ["nvcc", *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", LIB, *sources()]
+    cmd += ["-o", LIB, *sources(), "-ldl"]
     subprocess.run(cmd, check=True)
     return LIB
 

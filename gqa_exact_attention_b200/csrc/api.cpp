@@ -4,12 +4,14 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <dlfcn.h>
 
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
 #include <mutex>
+#include <string>
 #include <vector>
 
 #include "fwd_params.h"
@@ -126,8 +128,9 @@ int choose_splits_varlen(const Plan& pl, int d, int num_sms) {
     return s > dense ? s : dense;
 }
 
-// Tuned schedules, read once per process from the text file named by GQA_TUNE_TABLE (as
-// written by the package's autotune module).  One entry per line:
+// Tuned schedules, read once per process from the text file named by GQA_TUNE_TABLE, or
+// when that is unset from the table shipped beside the library (both as written by the
+// package's autotune module).  One entry per line:
 //   d causal Hq Hk bucket(B) bucket(Sq) bucket(Sk) pack_gqa num_splits [anything else]
 // with bucket(x) = the smallest e such that 2^e >= x.  '#' starts a comment line; lines
 // that do not parse are skipped; a later line for the same key wins.
@@ -141,13 +144,26 @@ int bucket(int x) {
     return e;
 }
 
+// The table shipped beside the library (tune_b200.txt in the directory of this shared
+// object), measured on B200 for the benchmark workloads.
+std::string default_table_path() {
+    Dl_info info{};
+    if (dladdr(reinterpret_cast<void*>(&gqa_attn_choose), &info) == 0 || info.dli_fname == nullptr)
+        return std::string();
+    const std::string so(info.dli_fname);
+    const size_t slash = so.find_last_of('/');
+    return (slash == std::string::npos ? std::string(".") : so.substr(0, slash)) + "/tune_b200.txt";
+}
+
 const std::vector<TuneEntry>& tune_table() {
     static std::vector<TuneEntry> table;
     static std::once_flag once;
     std::call_once(once, [] {
-        const char* path = std::getenv("GQA_TUNE_TABLE");
-        if (path == nullptr || *path == '\0') return;
-        FILE* f = std::fopen(path, "r");
+        // GQA_TUNE_TABLE names the table; set but empty, no table; unset, the shipped one
+        const char* env = std::getenv("GQA_TUNE_TABLE");
+        const std::string path = env != nullptr ? std::string(env) : default_table_path();
+        if (path.empty()) return;
+        FILE* f = std::fopen(path.c_str(), "r");
         if (f == nullptr) return;
         char line[512];
         while (std::fgets(line, sizeof line, f) != nullptr) {

@@ -115,14 +115,16 @@ GQA_API gqa_status gqa_attn_fwd(const void* q, const void* k, const void* v, flo
  * of a unit then end on the same key block), split the key axis when the (batch, head,
  * q-tile) units alone cannot fill the SMs.
  *
- * Tuned schedules replace the rule: if the environment variable GQA_TUNE_TABLE names a
- * table file (written by the package's autotune module; read once per process, at the
- * first call that needs it), a shape whose bucket (d, causal, Hq, Hk and the power-of-two
- * buckets of B, Sq, Sk) has an entry gets that entry's pack_gqa / num_splits, validated
- * for the shape (packing needs Hq/Hk <= 128; splits are clamped to the key blocks).
- * The same applies to gqa_attn_fwd called with pack_gqa = -1 and num_splits = 0; not to
- * gqa_attn_fwd_kvcache with per-sequence lengths.  A missing or unreadable file leaves
- * the rule in place.
+ * Tuned schedules replace the rule.  The table (written by the package's autotune module;
+ * read once per process, at the first call that needs it) is the file named by the
+ * environment variable GQA_TUNE_TABLE or, when that variable is unset, tune_b200.txt in the
+ * directory of this library: the table shipped with it, measured on B200 over the
+ * benchmark workloads.  GQA_TUNE_TABLE set to the empty string turns tuning off.  A shape
+ * whose bucket (d, causal, Hq, Hk and the power-of-two buckets of B, Sq, Sk) has an entry
+ * gets that entry's pack_gqa / num_splits, validated for the shape (packing needs
+ * Hq/Hk <= 128; splits are clamped to the key blocks).  The same applies to gqa_attn_fwd
+ * called with pack_gqa = -1 and num_splits = 0; not to gqa_attn_fwd_kvcache with
+ * per-sequence lengths.  A missing or unreadable file leaves the rule in place.
  */
 GQA_API gqa_status gqa_attn_choose(int B, int Sq, int Sk, int Hq, int Hk, int d, int causal,
                            int num_sms, int* pack_gqa, int* num_splits);

@@ -144,3 +144,31 @@ def test_other_scales(scale, causal, pack, splits):
     o_ref, l_ref = P.oracle_full(seed, *shp, scale, causal)
     out, lse = run(q, k, v, causal, pack, splits, scale=scale)
     P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"scale {scale} c{causal} p{pack} s{splits}")
+
+
+# --- short query axes (decode, a few positions): tiles with at most 32 real rows, every
+# pack/split schedule against the oracle and against nine splits.
+SHORT_Q = [
+    # B, Sq, Sk, Hq, Hk, d           real rows per tile (packed)
+    (4, 1, 3000, 32, 8, 128),        # g=4: 4
+    (2, 8, 1200, 32, 8, 128),        # 4 x 8 = 32, causal rows end at different keys
+    (2, 3, 1200, 30, 3, 64),         # g=10: 30, a quarter box of 3 positions
+    (1, 20, 1300, 4, 4, 64),         # MHA: 20 positions
+    (3, 1, 1153, 32, 1, 128),        # MQA g=32: 32; one key past the last full block
+]
+
+
+@pytest.mark.parametrize("shp", SHORT_Q, ids=[str(s) for s in SHORT_Q])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_short_query_axis_schedules(shp, causal):
+    seed = 3500 + sum(shp)
+    q, k, v = P.device_inputs(seed, *shp)
+    d = shp[5]
+    o_ref, l_ref = P.oracle_full(seed, *shp, P.default_scale(d), causal)
+    whole, lwhole = run(q, k, v, causal, 1, 9)
+    P.check(whole.cpu().numpy(), lwhole.cpu().numpy(), o_ref, l_ref, f"{shp} c{causal} p1 s9")
+    for pack, splits in ((-1, 0), (1, 1), (0, 1), (1, 3), (0, 8)):
+        out, lse = run(q, k, v, causal, pack, splits)
+        P.check(out.cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, f"{shp} c{causal} p{pack} s{splits}")
+        assert (out - whole).abs().max().item() <= P.VARIANT_MAX
+        assert (lse - lwhole).abs().max().item() <= P.VARIANT_MAX

@@ -20,9 +20,12 @@ print(json.dumps([list(G.gqa_attn_choose(*s)) for s in shapes]))
 
 
 def choose_with_table(table_text, shapes, tmp_path):
-    """gqa_attn_choose for each shape in a fresh process reading this table."""
+    """gqa_attn_choose for each shape in a fresh process reading this table (None: no
+    table, the heuristic; "shipped": GQA_TUNE_TABLE unset, the table beside the library)."""
     env = dict(os.environ)
     if table_text is None:
+        env["GQA_TUNE_TABLE"] = ""
+    elif table_text == "shipped":
         env.pop("GQA_TUNE_TABLE", None)
     else:
         path = tmp_path / "tune.txt"
@@ -89,3 +92,33 @@ def test_table_round_trip(tmp_path):
            T.key(32, 1, 8192, 32, 8, 128, 0): (1, 2, 0.17)}
     T.write_table(path, tab)
     assert T.read_table(path) == tab
+
+
+SHIPPED = os.path.join(ROOT, "gqa_exact_attention_b200", "tune_b200.txt")
+
+
+def test_shipped_table_is_read_by_default(tmp_path):
+    """With GQA_TUNE_TABLE unset the library reads the table shipped beside it; set to the
+    empty string, no table at all (the heuristic)."""
+    table = T.read_table(SHIPPED)
+    assert table, "the package ships a tuned table"
+    shapes = T.preset_workloads()
+    shipped = choose_with_table("shipped", shapes, tmp_path)
+    heur = choose_with_table(None, shapes, tmp_path)
+    for shp, got, h in zip(shapes, shipped, heur):
+        k = T.key(*shp)
+        assert k in table, f"{shp} is not in the shipped table"
+        blocks = -(-shp[2] // 128)
+        want = (table[k][0], min(table[k][1], blocks, 16))
+        assert got == want, (shp, got, want)
+    # the same table named explicitly gives the same answers
+    assert choose_with_table(open(SHIPPED).read(), shapes, tmp_path) == shipped
+    assert len(heur) == len(shipped)
+
+
+def test_shipped_table_entries_are_valid():
+    for k, (pack, splits, ms) in T.read_table(SHIPPED).items():
+        d, causal, Hq, Hk = k[:4]
+        assert d in (64, 128) and causal in (0, 1) and Hq % Hk == 0
+        assert pack in (0, 1) and 1 <= splits <= 16 and ms > 0
+        assert pack == 0 or 1 < Hq // Hk <= 128
