@@ -40,7 +40,7 @@ if ROOT not in sys.path:
 METRIC = "GQA fwd TFLOPS & tokens/s (Hq32 Hk8 d128 S2K, B16-256); decode HBM GB/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SRC = os.path.join(ROOT, "gqa_exact_attention_b200", "csrc", "fwd_sm100.cu")
+CSRC_DIR = os.path.join(ROOT, "gqa_exact_attention_b200", "csrc")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -88,8 +88,14 @@ def load_peaks():
 
 
 def kernel_hash():
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256[:16] over the library's sources (kernels, host plan and schedule, headers):
+    any change that can move the kernel's DRAM traffic invalidates the stored counters."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC_DIR)):
+        if name.endswith((".cu", ".cuh", ".cpp", ".h")):
+            with open(os.path.join(CSRC_DIR, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_for(workload_key, pack_gqa, num_splits):
