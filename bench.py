@@ -665,26 +665,38 @@ def run_sweep_kvcache(args, peaks):
         out = torch.empty((B, Sq, Hq, d), dtype=odt, device="cuda")
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
 
-        def step():
+        def step(st=stream):
             G.gqa_attn_fwd_kvcache(q, k, v, sl, out=out, lse=lse, causal=causal, num_splits=sp,
-                                   stream=stream)
+                                   stream=st)
         for _ in range(args.warmup):
             step()
         torch.cuda.synchronize()
+        graph = None
+        if args.graph:
+            # the call's launches (work order, forward, combine) captured once and replayed
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(torch.cuda.current_stream())
+            graph.replay()
+            torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
-            step()
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
         e1.record(stream)
         torch.cuda.synchronize()
         if G.gqa_attn_device_status(reset=True) != 0:
             raise SystemExit("an in-kernel bounded wait timed out")
         ms = e0.elapsed_time(e1) / args.steps
+        del graph
         keys = int(lens.sum())
         osz = 2 if dt == "bf16" else 4
         by = 2 * B * Sq * Hq * d + 2 * 2 * keys * Hk * d + osz * B * Sq * Hq * d + 4 * B * Hq * Sq
         fl = sum(flops(1, Sq, int(L), Hq, d, causal) for L in lens)
-        line = {"sweep": "kvcache", "B": B, "Sq": Sq, "Sk_capacity": Sk, "lengths": mix,
+        line = {"sweep": "kvcache", "graph": bool(args.graph), "B": B, "Sq": Sq, "Sk_capacity": Sk, "lengths": mix,
                 "num_splits": sp if sp > 0 else "auto",
                 "mean_length": round(float(lens.mean()), 1), "causal": bool(causal), "out": dt,
                 "ms": round(ms, 4), "hbm_gbs": round(by / ms / 1e6, 1),
@@ -849,6 +861,8 @@ def main():
                     help="skip the >= 1 s timed region of the main step")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the decode workload of the default line")
+    ap.add_argument("--graph", action="store_true",
+                    help="--sweep kvcache: replay each call from a CUDA graph")
     ap.add_argument("--sweep", choices=["prefill", "decode", "kvcache", "paged", "fp8"], default=None,
                     help="print one line per configuration of the batch sweep or decode grid")
     args = ap.parse_args()

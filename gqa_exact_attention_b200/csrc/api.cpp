@@ -434,6 +434,7 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     gqa_status st = validate_shape(B, Sq, paged ? 1 : Sk, Hq, Hk, d, pack_gqa, num_splits);
     if (st != GQA_OK) return st;
     if (paged != nullptr) {
+        if (f8 != nullptr) return GQA_ERR_SHAPE;  // no e4m3 page pools
         if (!paged->block_table || !seqlens_k) return GQA_ERR_NULL;
         if (!is_pow2(paged->page_size) || paged->page_size < 16 || paged->num_pages < 1 ||
             paged->table_stride < 1 ||
@@ -515,10 +516,16 @@ gqa_status fwd_impl(const void* q, const void* k, const void* v, const int* seql
     const double qk = is_f8 ? (double)f8->q_scale * (double)f8->k_scale : 1.0;
     p.scale_log2 = (float)((double)scale * qk * 1.4426950408889634);
     p.v_scale = is_f8 ? f8->v_scale : 1.f;
+    // readers of each K/V block: the query-tile units of a (batch, head-or-group), times the
+    // heads of a group when they are not packed together
+    p.kv_shared = ((long long)pl.n_mt * (pl.pack ? 1 : g) > 1) ? 1 : 0;
     p.div_g = gqa::make_fastdiv((uint32_t)g);
     p.status = nullptr;
     p.timeout_ns = timeout_ns();
     p.drain_ns = drain_ns(p.timeout_ns);
+    // host-side fault injection: the kernel stalls on a wait that nothing completes and
+    // reports GQA_ERR_TIMEOUT through the status word (tests of the bounded waits)
+    p.inject_stall = std::getenv("GQA_FAULT_INJECT_STALL") != nullptr ? 1 : 0;
 
     // Device scratch: the split partials (num_splits > 1), and with per-sequence lengths the
     // work order of the units (2 ints per unit), in one stream-ordered pool allocation, or

@@ -68,6 +68,13 @@ struct FwdParams {
     // e4m3 inputs: V's per-tensor scale, applied to O in the epilogue (1 for bf16 inputs;
     // Q's and K's scales are folded into scale_log2)
     float v_scale;
+    // K/V blocks are read by more than one unit (several query tiles, or unpacked heads,
+    // per kv-head): their loads then ask L2 to keep them (evict_last); else they stream
+    // (evict_first), like the Q tiles always do
+    int kv_shared;
+    // fault injection for the failure-detection tests: the producer first waits on a barrier
+    // that nothing arrives on, so that the wait limit runs out (GQA_FAULT_INJECT_STALL)
+    int inject_stall;
 };
 
 struct CombineParams {

@@ -87,7 +87,7 @@ struct FwdCfg {
     // blocks only); the rest use the special-function unit
     static constexpr int kPolyPairs = GQA_EXP_POLY_PAIRS;
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
-    static constexpr int kNumBars = 2 * kSlots + 8 * NT + 1;
+    static constexpr int kNumBars = 2 * kSlots + 8 * NT + 2;
     static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
     // epilogue staging for TMA stores: 128 rows x 32 fp32 (128 B, swizzled) per chunk
     static constexpr int kOStageBytes = kEpilogueWG ? 128 * 128 : 0;
@@ -303,26 +303,13 @@ __device__ __forceinline__ int page_of(PageCache& pc, const FwdParams& p, int b,
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting or when
 // this wait ran past the time limit (then it records the timeout and starts the abort).
-// Normal limits: suspending probes (try_wait), the clock and the abort flag read every 256
-// of them.  Limits under 100 us exist only to exercise this path; a suspending probe can
-// cover a whole wait of several microseconds by itself, so those use non-suspending probes
-// (test_wait) and read the clock at every probe, and a wait of a few microseconds
-// reliably runs out.
+// Suspending probes (try_wait); the clock and the abort flag are read every 256 of them.
+// The code inlined at each wait site is kept this small on purpose: a larger inlined wait
+// (a second, test-only probe loop) measured 4-7 % slower prefill, the hot loops' code
+// sharing the SM's instruction cache with every wait site.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile uint32_t* abort_flag,
                                              const FwdParams& p) {
-    if (p.timeout_ns < 100000) {
-        const uint64_t t0 = globaltimer();
-        while (!mbar_test_wait(bar, parity)) {
-            if (*abort_flag) return false;
-            if ((long long)(globaltimer() - t0) > p.timeout_ns) {
-                *abort_flag = 1u;
-                atomicOr(p.status ? p.status : &g_device_status, 1u);
-                return false;
-            }
-        }
-        return true;
-    }
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer();
     uint32_t spins = 0;
@@ -349,7 +336,10 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, const 
     }
 }
 
-template <int HD, int NT, bool F8>
+// PAGED: K/V come from page pools through the block table (the producer's address
+// computation only; a separate instantiation, so the dense kernels carry none of it in
+// their instruction stream).
+template <int HD, int NT, bool F8, bool PAGED>
 __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F8>::kCtasPerSm)
     gqa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = FwdCfg<HD, NT, F8>;
@@ -382,6 +372,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
     // the next post needs the epilogue to have released O_t of the unit before.
     auto st_full = [&](int t, uint32_t buf) { return bar0 + 8u * (2 * C::kSlots + 6 * NT + 2 * t + buf); };
     const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 8 * NT);
+    // never arrived on: the injected stall waits on it (failure-detection tests)
+    const uint32_t stall_bar = bar0 + 8u * (2 * C::kSlots + 8 * NT + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -403,6 +395,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
             mbar_init(st_full(t, 1), 128);
         }
         mbar_init(mma_done, 1);
+        mbar_init(stall_bar, 1);
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -442,12 +435,16 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                     const int hcoord = p.pack ? g.hg * p.g : g.hg;
 #pragma unroll
                     for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_4d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
-                                    q_full(t), c * 64, hcoord, g.pos0[t], g.b);
+                        tma_load_4d_hint(sQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
+                                         q_full(t), c * 64, hcoord, g.pos0[t], g.b,
+                                         l2_policy_evict_first());
                 }
                 __syncwarp();
                 ++qn[t];
             };
+            // Injected stall (failure-detection tests): a wait that nothing completes runs
+            // out at the wait limit and aborts the CTA, as a copy that never lands would.
+            if (p.inject_stall) ok = __all_sync(0xffffffffu, wait_bounded(stall_bar, 0u, abort_flag, p));
             // Load order per unit: Q_0, K_0, Q_1.., V_0, K_1, V_1, ...  The MMA warp may
             // issue a unit's first S_0 while the unit before still runs on tile 1, so K_0
             // must not queue behind Q_1 (which waits for that unit's last S_1).
@@ -460,9 +457,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                     // page row range each); sub-ranges at or past this sequence's key count
                     // take a page coordinate past the pool, which TMA fills with zeros
                     // (masked anyway), so no table entry past the sequence is used
-                    int pg[8], prow[8];
-                    const int nsub = p.block_table ? kBlockN / p.page_rows : 1;
-                    if (p.block_table) {
+                    [[maybe_unused]] int pg[8], prow[8];
+                    [[maybe_unused]] const int nsub = PAGED ? kBlockN / p.page_rows : 1;
+                    if constexpr (PAGED) {
 #pragma unroll
                         for (int sub = 0; sub < 8; ++sub) {
                             if (sub >= nsub) break;
@@ -481,20 +478,22 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                         if (elect_one()) {
                             mbar_arrive_expect_tx(kv_full(slot), (uint32_t)C::kTileBytes);
                             const void* tm = w == 0 ? (const void*)&p.tm_k : (const void*)&p.tm_v;
-                            if (p.block_table == nullptr) {
+                            const uint64_t pol = p.kv_shared ? l2_policy_evict_last() : l2_policy_evict_first();
+                            if constexpr (!PAGED) {
 #pragma unroll
                                 for (int c = 0; c < C::kChunks; ++c)
-                                    tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes, tm,
-                                                kv_full(slot), c * 64, g.kvh, kpos, g.b);
+                                    tma_load_4d_hint(sKV + slot * C::kTileBytes + c * C::kChunkBytes, tm,
+                                                     kv_full(slot), c * 64, g.kvh, kpos, g.b, pol);
                             } else {
 #pragma unroll
                                 for (int sub = 0; sub < 8; ++sub) {
                                     if (sub >= nsub) break;
 #pragma unroll
                                     for (int c = 0; c < C::kChunks; ++c)
-                                        tma_load_4d(sKV + slot * C::kTileBytes + c * C::kChunkBytes +
-                                                        sub * p.page_rows * C::kChunkRowBytes,
-                                                    tm, kv_full(slot), c * 64, g.kvh, prow[sub], pg[sub]);
+                                        tma_load_4d_hint(sKV + slot * C::kTileBytes + c * C::kChunkBytes +
+                                                             sub * p.page_rows * C::kChunkRowBytes,
+                                                         tm, kv_full(slot), c * 64, g.kvh, prow[sub],
+                                                         pg[sub], pol);
                                 }
                             }
                         }
@@ -1036,7 +1035,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                             fence_proxy_async_smem();
                             named_bar_sync(kEpiBar, 128);
                             if (issuer) {
-                                tma_store_4d(&p.tm_o, sO, (ch >> 1) * 64, hcoord, g.pos0[t], bcoord);
+                                tma_store_4d_hint(&p.tm_o, sO, (ch >> 1) * 64, hcoord, g.pos0[t], bcoord,
+                                                  l2_policy_evict_first());
                                 bulk_commit_group();
                             }
                         }
@@ -1074,7 +1074,13 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                     fence_proxy_async_smem();
                     named_bar_sync(kEpiBar, 128);
                     if (issuer) {
-                        tma_store_4d(&p.tm_o, sO, ch * 32, hcoord, g.pos0[t], bcoord);
+                        // the final output is not read again here; split partials are,
+                        // by the combine, and keep the default policy
+                        if (p.num_splits == 1)
+                            tma_store_4d_hint(&p.tm_o, sO, ch * 32, hcoord, g.pos0[t], bcoord,
+                                              l2_policy_evict_first());
+                        else
+                            tma_store_4d(&p.tm_o, sO, ch * 32, hcoord, g.pos0[t], bcoord);
                         bulk_commit_group();
                     }
                 }
@@ -1215,7 +1221,7 @@ __global__ void __launch_bounds__(256) gqa_combine_kernel(const CombineParams p)
     }
 }
 
-template <int HD, int NT, bool F8>
+template <int HD, int NT, bool F8, bool PAGED>
 cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
     using C = FwdCfg<HD, NT, F8>;
     // the attribute is per device; setting it again is idempotent, so the race is benign
@@ -1223,7 +1229,7 @@ cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(gqa_fwd_kernel<HD, NT, F8>,
+        cudaError_t e = cudaFuncSetAttribute(gqa_fwd_kernel<HD, NT, F8, PAGED>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kSmemBytes);
         if (e != cudaSuccess) return e;
@@ -1234,12 +1240,12 @@ cudaError_t launch_fwd_t(const FwdParams& p, int grid, cudaStream_t stream) {
     static int regs_checked = 0;  // 0 unknown, 1 ok, -1 mismatch
     if (regs_checked == 0) {
         cudaFuncAttributes attr{};
-        cudaError_t e = cudaFuncGetAttributes(&attr, gqa_fwd_kernel<HD, NT, F8>);
+        cudaError_t e = cudaFuncGetAttributes(&attr, gqa_fwd_kernel<HD, NT, F8, PAGED>);
         if (e != cudaSuccess) return e;
         regs_checked = (attr.numRegs == C::kLaunchRegs) ? 1 : -1;
     }
     if (regs_checked != 1) return cudaErrorInvalidConfiguration;
-    gqa_fwd_kernel<HD, NT, F8><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
+    gqa_fwd_kernel<HD, NT, F8, PAGED><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -1252,11 +1258,15 @@ int fwd_ctas_per_sm(int hd, int nt) {
 
 cudaError_t launch_fwd(const FwdParams& p, int hd, int nt, bool f8, int grid, cudaStream_t stream) {
     if (f8) {
-        if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, true>(p, grid, stream) : launch_fwd_t<128, 1, true>(p, grid, stream);
-        return nt == 2 ? launch_fwd_t<64, 2, true>(p, grid, stream) : launch_fwd_t<64, 1, true>(p, grid, stream);
+        if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, true, false>(p, grid, stream) : launch_fwd_t<128, 1, true, false>(p, grid, stream);
+        return nt == 2 ? launch_fwd_t<64, 2, true, false>(p, grid, stream) : launch_fwd_t<64, 1, true, false>(p, grid, stream);
     }
-    if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, false>(p, grid, stream) : launch_fwd_t<128, 1, false>(p, grid, stream);
-    return nt == 2 ? launch_fwd_t<64, 2, false>(p, grid, stream) : launch_fwd_t<64, 1, false>(p, grid, stream);
+    if (p.block_table != nullptr) {
+        if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, false, true>(p, grid, stream) : launch_fwd_t<128, 1, false, true>(p, grid, stream);
+        return nt == 2 ? launch_fwd_t<64, 2, false, true>(p, grid, stream) : launch_fwd_t<64, 1, false, true>(p, grid, stream);
+    }
+    if (hd == 128) return nt == 2 ? launch_fwd_t<128, 2, false, false>(p, grid, stream) : launch_fwd_t<128, 1, false, false>(p, grid, stream);
+    return nt == 2 ? launch_fwd_t<64, 2, false, false>(p, grid, stream) : launch_fwd_t<64, 1, false, false>(p, grid, stream);
 }
 
 cudaError_t launch_unit_order(const FwdParams& p, int nt, int grid, int* order, int* tmp,

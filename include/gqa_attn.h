@@ -274,7 +274,9 @@ GQA_API const char* gqa_attn_status_string(gqa_status status);
  * tensor memory and exits; the rest of the grid notices and exits the same way.  The
  * call itself has already returned GQA_OK (it is asynchronous), and out / lse are then
  * partly unwritten: read this word after synchronising when that matters.  Later calls
- * are unaffected.
+ * are unaffected.  With GQA_FAULT_INJECT_STALL set (tests of this path), every CTA first
+ * waits on a barrier that nothing completes, so the limit runs out on purpose; the GPU
+ * stays healthy and the next call without it runs normally.
  */
 GQA_API gqa_status gqa_attn_device_status(int reset);
 

@@ -6,14 +6,15 @@ Two paths, each driven by the library's own host-side switches:
   fail as it would on an exhausted device.  The call must return GQA_ERR_ALLOC before
   launching anything (out and lse keep their NaN fill); calls that need no allocation
   still run.
-* Bounded waits.  Every wait inside the forward kernel is bounded.  With the limit set
-  to 100 ns (GQA_WAIT_TIMEOUT_NS), the kernel's ordinary waits for copies and MMAs run
-  out.  The call must still return (asynchronously, GQA_OK), the device status word must
-  read GQA_ERR_TIMEOUT after synchronising, and a normal call afterwards must match the
-  oracle.  Nothing is withheld or broken: only the limit is short.  This runs in a child
-  process under a time limit, once for the one-tile kernel (decode-like shape, the
-  softmax warpgroup writes the output) and once for the two-tile kernel (prefill-like
-  shape, epilogue warpgroup with TMA stores).
+* Bounded waits.  Every wait inside the forward kernel is bounded.  GQA_FAULT_INJECT_STALL
+  makes each CTA first wait on a barrier that nothing arrives on (a flag that nothing
+  sets), with the limit at 20 ms (GQA_WAIT_TIMEOUT_MS).  The call must still return
+  (asynchronously, GQA_OK), the device status word must read GQA_ERR_TIMEOUT after
+  synchronising, every other warp must notice the abort and exit, and a normal call
+  afterwards must match the oracle.  This runs in a child process under a time limit,
+  once for the one-tile kernel (decode-like shape, the softmax warpgroup writes the
+  output) and once for the two-tile kernel (prefill-like shape, epilogue warpgroup with
+  TMA stores).
 """
 import json
 import os
@@ -91,14 +92,16 @@ seed = 7200 + Sq
 q, k, v = P.device_inputs(seed, *shp)
 res = {}
 assert G.gqa_attn_device_status(reset=True) == 0
-os.environ["GQA_WAIT_TIMEOUT_NS"] = "100"
+os.environ["GQA_WAIT_TIMEOUT_MS"] = "20"
+os.environ["GQA_FAULT_INJECT_STALL"] = "1"
 t0 = time.time()
 out, lse = G.gqa_attn_fwd(q, k, v, pack_gqa=pack, num_splits=splits)  # returns: async
 res["returned"] = True
 torch.cuda.synchronize()
 res["sync_s"] = time.time() - t0
 res["status_after_short_limit"] = G.gqa_attn_device_status(reset=True)
-del os.environ["GQA_WAIT_TIMEOUT_NS"]
+del os.environ["GQA_FAULT_INJECT_STALL"]
+del os.environ["GQA_WAIT_TIMEOUT_MS"]
 out, lse = G.gqa_attn_fwd(q, k, v, pack_gqa=pack, num_splits=splits)
 torch.cuda.synchronize()
 res["status_after_normal_call"] = G.gqa_attn_device_status(reset=True)
@@ -114,8 +117,8 @@ print("RESULT " + json.dumps(res), flush=True)
 ], ids=["one_tile", "two_tiles"])
 def test_bounded_wait_timeout_is_reported_and_recoverable(shp, pack, splits):
     env = dict(os.environ)
-    env.pop("GQA_WAIT_TIMEOUT_NS", None)
-    env.pop("GQA_WAIT_TIMEOUT_MS", None)
+    for name in ("GQA_WAIT_TIMEOUT_NS", "GQA_WAIT_TIMEOUT_MS", "GQA_FAULT_INJECT_STALL"):
+        env.pop(name, None)
     r = subprocess.run([sys.executable, "-c", _CHILD, json.dumps(list(shp)), str(pack), str(splits)],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
