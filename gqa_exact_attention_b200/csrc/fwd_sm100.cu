@@ -1130,12 +1130,42 @@ __global__ void __launch_bounds__(1024) gqa_unit_order_kernel(const __grid_const
     };
     for (int u = threadIdx.x; u < p.n_units; u += blockDim.x) atomicAdd(&cnt[bucket_of(u)], 1);
     __syncthreads();
-    if (threadIdx.x == 0) {  // exclusive prefix sum (2048 entries, once)
-        int acc = 0;
-        for (int i = 0; i < kBuckets; ++i) {
-            const int c = cnt[i];
-            cnt[i] = acc;
-            acc += c;
+    // exclusive prefix sum of the counts: each of the 1024 threads owns kPer consecutive
+    // buckets; warp shuffles scan the threads' totals, one warp scans the warps' totals
+    {
+        constexpr int kPer = kBuckets / 1024;
+        __shared__ int warp_sum[32];
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        int own[kPer];
+        int tot = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            own[j] = cnt[threadIdx.x * kPer + j];
+            tot += own[j];
+        }
+        int incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_sum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int w = warp_sum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sum[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        int base = incl - tot + (warp > 0 ? warp_sum[warp - 1] : 0);
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            cnt[threadIdx.x * kPer + j] = base;
+            base += own[j];
         }
     }
     __syncthreads();
