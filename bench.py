@@ -599,7 +599,7 @@ def run_sweep(args):
                  for (pk, sp) in [(-1, 0), (1, 1), (1, 2), (1, 4), (1, 8)]]
     cur = None
     for (B, Sq, Sk, causal, pk, sp) in cases:
-        Hq, Hk, d = 32, 8, 128
+        Hq, Hk, d = 32, 8, args.d
         if cur != (B, Sq, Sk):
             q = k = v = out = lse = None
             torch.cuda.empty_cache()
@@ -626,7 +626,7 @@ def run_sweep(args):
         ms = e0.elapsed_time(e1) / args.steps
         fl = flops(B, Sq, Sk, Hq, d, causal)
         by = hbm_bytes(B, Sq, Sk, Hq, Hk, d)
-        line = {"sweep": args.sweep, "B": B, "Sq": Sq, "Sk": Sk, "causal": bool(causal),
+        line = {"sweep": args.sweep, "B": B, "Sq": Sq, "Sk": Sk, "d": d, "causal": bool(causal),
                 "pack_gqa": rp, "num_splits": rs, "heuristic": pk < 0 and sp <= 0,
                 "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1),
                 "hbm_gbs": round(by / ms / 1e6, 1),
