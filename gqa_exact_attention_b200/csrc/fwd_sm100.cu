@@ -29,8 +29,13 @@
 #include "exp2_poly.cuh"
 #include "ptx_sm100.cuh"
 
-#ifndef GQA_EXP_POLY_PAIRS
-#define GQA_EXP_POLY_PAIRS 4
+// Of each 16 exponential pairs of an unmasked 32-key chunk, how many take the FMA-pipe
+// polynomial instead of the MUFU; measured per head dimension on B200 (interleaved timing
+// of 2-6 pairs): 2 at d=128, 3 at d=64.  -DGQA_EXP_POLY_PAIRS=n overrides both.
+#ifdef GQA_EXP_POLY_PAIRS
+#define GQA_POLY_PAIRS_FOR(HD) (GQA_EXP_POLY_PAIRS)
+#else
+#define GQA_POLY_PAIRS_FOR(HD) ((HD) == 128 ? 2 : 3)
 #endif
 
 namespace gqa {
@@ -85,7 +90,7 @@ struct FwdCfg {
                   "epilogue registers");
     // of each 16 exponential pairs of a 32-key chunk, this many take the polynomial (unmasked
     // blocks only); the rest use the special-function unit
-    static constexpr int kPolyPairs = GQA_EXP_POLY_PAIRS;
+    static constexpr int kPolyPairs = GQA_POLY_PAIRS_FOR(HD);
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
     static constexpr int kNumBars = 2 * kSlots + 8 * NT + 2;
     static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
