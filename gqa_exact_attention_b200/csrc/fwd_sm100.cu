@@ -1,16 +1,22 @@
 // Exact GQA attention forward for sm_100a: persistent, warp-specialised, TMA + tcgen05.
 //
-// One CTA runs on one SM and walks a static stride of work units.  A unit is NT
-// consecutive 128-row query tiles of one (batch, head) pair (or, with PackGQA, of one
-// (batch, kv-group) pair whose g query heads are folded into the rows), over one
-// split of the key axis.  Roles:
-//   warp 0        TMA producer: Q tiles once per unit, then a ring of K/V blocks.
-//   warp 1        MMA issuer (one thread): S_t = Q_t K^T into TMEM (both operands in
-//                 shared memory), then O_t += P_t V with P_t read from TMEM.
-//   warps 2..     NT softmax warpgroups, one per tile; thread = tile row = TMEM lane.
-//                 Each reads its S row from TMEM, masks (causal, key tail), keeps the
-//                 running max / sum, writes P (bf16) over S in TMEM, rescales O in TMEM
-//                 when the max grows, and runs the epilogue (O / l, LSE).
+// Persistent CTAs walk a static stride of work units: one CTA per SM for two-tile
+// units (NT = 2, prefill), two per SM for one-tile units (NT = 1, decode and short query
+// axes).  A unit is NT consecutive 128-row query tiles of one (batch, head) pair (or,
+// with PackGQA, of one (batch, kv-group) pair whose g query heads are folded into the
+// rows), over one split of the key axis.  Roles:
+//   warpgroup 0, warp 0   TMA producer: Q tiles once per unit, then a ring of K/V blocks
+//                         (a page pool through the block table in the PAGED kernels).
+//   warpgroup 0, warp 1   MMA issuer, a converged warp whose elected lane issues:
+//                         S_t = Q_t K^T into TMEM (both operands in shared memory), then
+//                         O_t += P_t V with P_t read from TMEM.
+//   warpgroups 1..NT      softmax, one per tile; thread = tile row = TMEM lane.  Each
+//                         reads its S row from TMEM, masks (causal, key tail), keeps the
+//                         reference max and row sum, writes P (bf16 or e4m3) over S in
+//                         TMEM and rescales O in TMEM when the reference max moves.
+//   warpgroup NT + 1      (NT = 2 only) epilogue: O / l through a shared-memory stage and
+//                         TMA tensor stores, and the LSE.  With NT = 1 the softmax
+//                         warpgroup writes its rows' output itself.
 //
 // The computation follows the scaled dot-product attention definition
 // ("PyTorch 性能分析深度指南 (第三部分)", section "Attention 的计算挑战") with the GQA head
