@@ -80,3 +80,19 @@ def test_committed_traffic_matches_the_current_kernel(bench):
     w = t["workloads"]["prefill B=64 Hq=32 Hk=8 Sq=Sk=2048 d=128 causal"]
     assert w["algorithmic_bytes"] == bench.hbm_bytes(64, 2048, 2048, 32, 8, 128)
     assert w["dram_bytes_per_launch"] == w["dram_bytes_read"] + w["dram_bytes_write"]
+
+
+def test_committed_traffic_covers_both_objects_of_the_default_line(bench):
+    """The default line reports roofline.traffic for the prefill workload and for its
+    decode object; the committed counters must be found under both names (and agree with
+    the algorithmic accounting), or a matching source hash would still print null."""
+    t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    if t["kernel_sha256_16"] != bench.kernel_hash():
+        pytest.skip("the counters are for an earlier kernel source: the bench reports null")
+    c = bench.DECODE_CFG
+    for name, shape in (("prefill B=64 Hq=32 Hk=8 Sq=Sk=2048 d=128 causal", (64, 2048, 2048, 32, 8, 128)),
+                        (c["name"], (c["B"], c["Sq"], c["Sk"], c["Hq"], c["Hk"], c["d"]))):
+        assert bench.traffic_for(name, 1, 1) is not None, name
+        w = t["workloads"][name]
+        assert w["algorithmic_bytes"] == bench.hbm_bytes(*shape)
+        assert 0.9 < w["dram_bytes_per_launch"] / w["algorithmic_bytes"] < 1.3
