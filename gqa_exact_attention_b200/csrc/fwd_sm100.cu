@@ -14,6 +14,10 @@
 //                         reads its S row from TMEM, masks (causal, key tail), keeps the
 //                         reference max and row sum, writes P (bf16 or e4m3) over S in
 //                         TMEM and rescales O in TMEM when the reference max moves.
+//                         At d = 64 with two bf16 tiles, P has TMEM columns of its own
+//                         (S and O use 384 of 512), so the MMA issuer starts the next
+//                         block's S as soon as the softmax holds this block's S in
+//                         registers, ahead of this block's P.V.
 //   warpgroup NT + 1      (NT = 2 only) epilogue: O / l through a shared-memory stage and
 //                         TMA tensor stores, and the LSE.  With NT = 1 the softmax
 //                         warpgroup writes its rows' output itself.
@@ -98,7 +102,12 @@ struct FwdCfg {
     // blocks only); the rest use the special-function unit
     static constexpr int kPolyPairs = GQA_POLY_PAIRS_FOR(HD);
     static constexpr int kTmemCols = (NT * 128 + NT * HD) <= 256 ? 256 : 512;
-    static constexpr int kNumBars = 2 * kSlots + 8 * NT + 2;
+    // d=64 with two tiles (bf16): S and O take 384 of TMEM's 512 columns, which leaves room
+    // for P in columns of its own.  The next block's S is then computed while this block's
+    // softmax still runs (it needs only the S values already in registers), instead of
+    // after this block's P.V.
+    static constexpr bool kSepP = (HD == 64 && NT == 2 && !F8);
+    static constexpr int kNumBars = 2 * kSlots + 8 * NT + 2 + (kSepP ? 2 * NT : 0);
     static constexpr int kStatsBytes = kEpilogueWG ? 2 * NT * 2 * 128 * 4 : 0;  // (m, l), 2 buffers
     // epilogue staging for TMA stores: 128 rows x 32 fp32 (128 B, swizzled) per chunk
     static constexpr int kOStageBytes = kEpilogueWG ? 128 * 128 : 0;
@@ -121,6 +130,11 @@ struct FwdCfg {
     }
     __host__ __device__ static constexpr int s_col(int t) { return t * 128; }
     __host__ __device__ static constexpr int o_col(int t) { return NT * 128 + t * HD; }
+    __host__ __device__ static constexpr int p_col(int t) {
+        return kSepP ? NT * 128 + NT * HD + t * 64 : s_col(t);
+    }
+    // separate P sits this many columns past the tile's O (the same for every tile)
+    static constexpr int kPAfterO = NT * HD;
 };
 
 template <uint32_t R>
@@ -385,6 +399,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
     const uint32_t mma_done = bar0 + 8u * (2 * C::kSlots + 8 * NT);
     // never arrived on: the injected stall waits on it (failure-detection tests)
     const uint32_t stall_bar = bar0 + 8u * (2 * C::kSlots + 8 * NT + 1);
+    // separate P (kSepP): S_t read into registers (softmax -> MMA), P_t.V done (MMA -> softmax)
+    [[maybe_unused]] auto s_free = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 8 * NT + 2 + t); };
+    [[maybe_unused]] auto p_free = [&](int t) { return bar0 + 8u * (2 * C::kSlots + 8 * NT + 2 + NT + t); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -407,6 +424,12 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
         }
         mbar_init(mma_done, 1);
         mbar_init(stall_bar, 1);
+        if constexpr (C::kSepP) {
+            for (int t = 0; t < NT; ++t) {
+                mbar_init(s_free(t), 128);
+                mbar_init(p_free(t), 1);
+            }
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -562,7 +585,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                                 uint32_t probe_par) {
                 const uint64_t b0 = sdesc_add(v_desc0, slot * C::kTileBytes);
                 const uint32_t d = tmem + C::o_col(t);
-                const uint32_t a = tmem + C::s_col(t);
+                const uint32_t a = tmem + C::p_col(t);
                 bool ready = false;
                 if (elect_one()) {
                     // 8 TMEM columns of P per MMA (16 bf16 or 32 e4m3 keys)
@@ -583,6 +606,78 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                 return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p));
             };
 
+            if constexpr (C::kSepP) {
+            // Separate P: per key block, first S of the next block for every tile (once its
+            // softmax has taken this block's S into registers), then P.V of this block.
+            uint32_t sf[NT] = {};
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const UnitGeom<NT> g = unit_geom<NT>(u, p);
+                if (g.nblk == 0) continue;
+                int slot_k = ld % C::kSlots;
+                ok = wait(kv_full(slot_k), (ld / C::kSlots) & 1u);
+                if (!ok) break;
+                ++ld;
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (g.n[t] == 0 || !ok) continue;
+                    ok = wait(q_full(t), qn[t] & 1u);
+                    if (!ok) break;
+                    ++qn[t];
+                    tc_fence_after();
+                    issue_s(t, slot_k, 0u, 0u);
+                    commit(s_full(t));
+                    if (g.n[t] == 1) commit(q_empty(t));
+                }
+                if (!ok) break;
+                commit(kv_empty(slot_k));
+                for (int it = 0; it < g.nblk && ok; ++it) {
+                    const int slot_v = ld % C::kSlots;
+                    ok = wait(kv_full(slot_v), (ld / C::kSlots) & 1u);
+                    if (!ok) break;
+                    ++ld;
+                    if (it + 1 < g.nblk) {
+                        const int slot_n = ld % C::kSlots;
+                        ok = wait(kv_full(slot_n), (ld / C::kSlots) & 1u);
+                        if (!ok) break;
+                        ++ld;
+#pragma unroll
+                        for (int t = 0; t < NT; ++t) {
+                            if (it + 1 >= g.n[t] || !ok) continue;
+                            ok = wait(s_free(t), sf[t] & 1u);
+                            if (!ok) break;
+                            ++sf[t];
+                            tc_fence_after();
+                            issue_s(t, slot_n, 0u, 0u);
+                            commit(s_full(t));
+                            if (it + 2 == g.n[t]) commit(q_empty(t));
+                        }
+                        if (!ok) break;
+                        commit(kv_empty(slot_n));
+                    }
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        if (it >= g.n[t] || !ok) continue;
+                        ok = wait(p_full(t), pn[t] & 1u);
+                        if (!ok) break;
+                        ++pn[t];
+                        if (it == 0 && on[t] > 0) {
+                            // the previous unit's epilogue must have read O_t out
+                            ok = wait(o_empty(t), (on[t] - 1) & 1u);
+                            if (!ok) break;
+                        }
+                        tc_fence_after();
+                        issue_pv(t, slot_v, it > 0, 0u, 0u);
+                        commit(p_free(t));
+                        if (it + 1 == g.n[t]) {
+                            commit(o_full(t));
+                            ++on[t];
+                        }
+                    }
+                    if (!ok) break;
+                    commit(kv_empty(slot_v));
+                }
+            }
+            } else {
             // A tile that finishes its unit starts the next unit at once: its first S_t is
             // issued right after its last PV_t (the tensor pipe runs MMAs in issue order,
             // so S_t may overwrite the P_t that PV_t reads), instead of after every tile's
@@ -703,6 +798,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
 #pragma unroll
                 for (int t = 0; t < NT; ++t) early[t] = early_next[t];
             }
+            }
             // every MMA issued so far must be complete before TMEM is released
             commit(mma_done);
             wait_drain(mma_done, 0u, p);
@@ -716,6 +812,11 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
         const int row = quarter * 32 + lane;
         const uint32_t s_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::s_col(t);
         const uint32_t o_addr = tmem + ((uint32_t)(quarter * 32) << 16) + C::o_col(t);
+        static_assert(!C::kSepP || (C::p_col(0) - C::o_col(0) == C::kPAfterO &&
+                                    C::p_col(NT - 1) - C::o_col(NT - 1) == C::kPAfterO),
+                      "separate P lies a fixed distance past O");
+        // P's columns: S's own, or (separate P) a fixed distance past O's
+        const uint32_t p_addr = C::kSepP ? o_addr + C::kPAfterO : s_addr;
         const float c = p.scale_log2;
         const float kNegInf = -INFINITY;
         const float fill = (c >= 0.f) ? -INFINITY : INFINITY;  // masked keys drop out of the extremum
@@ -743,6 +844,18 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                     ++sn;
                     tc_fence_after();
                     tc_fence_before();
+                    if constexpr (C::kSepP) {
+                        if (it + 1 < n_t) mbar_arrive(s_free(t));
+                        // The next S may already be issued, so this warp could reach the
+                        // next block before the others finish this block's P: its early
+                        // arrivals would then complete this block's p_full.  Waiting for
+                        // the previous P.V keeps one arrival per thread per phase.
+                        // sn - 1 blocks of this tile came before this one
+                        if (sn > 1) {
+                            ok = __all_sync(0xffffffffu, wait_bounded(p_free(t), sn & 1u, abort_flag, p));
+                            if (!ok) break;
+                        }
+                    }
                     mbar_arrive(p_full(t));
                 }
                 if (!ok) break;
@@ -775,6 +888,13 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                     for (int i = 0; i < 32; ++i) s[ch * 32 + i] = __uint_as_float(r[i]);
                 }
                 tmem_wait_ld();
+                if constexpr (C::kSepP) {
+                    // S is in registers: the next block's S may be written over it
+                    if (it + 1 < n_t) {
+                        tc_fence_before();
+                        mbar_arrive(s_free(t));
+                    }
+                }
                 const int lim = kmax - (g.kb_lo + it) * kBlockN;  // keys [0, lim) allowed
                 // Warp-uniform view of the mask, per 32-key chunk: every key allowed for all
                 // 32 rows of the warp (full), none allowed for any of them (empty), or in
@@ -866,9 +986,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                         uint32_t q8[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) q8[i] = pk[i];
-                        tmem_st8(s_addr + ch * C::kPColsPer32, q8);
+                        tmem_st8(p_addr + ch * C::kPColsPer32, q8);
                     } else {
-                        tmem_st16(s_addr + ch * C::kPColsPer32, pk);
+                        tmem_st16(p_addr + ch * C::kPColsPer32, pk);
                     }
                 };
                 // one 32-key chunk: P = 2^(c s - m) as bf16 pairs; with kSelect, keys at or
@@ -922,6 +1042,15 @@ __global__ void __launch_bounds__(FwdCfg<HD, NT, F8>::kThreads, FwdCfg<HD, NT, F
                         }
                     }
                 };
+                if constexpr (C::kSepP) {
+                    // the previous block's P.V must be done before P and O are written again
+                    // P.V of block sn - 2 (this tile's previous one, if any)
+                    if (sn > 1) {
+                        ok = __all_sync(0xffffffffu, wait_bounded(p_free(t), sn & 1u, abort_flag, p));
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                }
                 if (masked) exp_range(std::true_type{}, 0, 2);
                 else exp_range(std::false_type{}, 0, 2);
                 // O rescale: PV of the previous block is complete, because this block's S
