@@ -1,5 +1,6 @@
-"""A discrete-event model of the hand-offs between the MMA warp and the softmax warps of one
-CTA of the two-tile forward kernel, for checking its barrier protocol on the CPU.
+"""A discrete-event model of one CTA of the two-tile forward kernel, for checking its barrier
+protocol on the CPU: the TMA producer, the MMA warp, four softmax warps per tile and the
+epilogue, with the hand-offs between them.
 
 What it models, in the kernel's terms:
 
@@ -7,18 +8,28 @@ What it models, in the kernel's terms:
   phase of that parity has completed, i.e. while the current phase's parity differs from
   it (the PTX ``mbarrier.try_wait.parity`` rule).  Arrivals that spill into a later phase,
   and a waiter that falls two phases behind, are what this model exists to catch.
+* TMA loads land in any order, each at a moment the scheduler picks, and arrive on their
+  full barrier.  Q_t has a buffer per tile; K and V blocks share a ring of slots, loaded in
+  the order Q_0, K_0, Q_1, V_0, K_1, V_1, ... per unit.
 * the tensor pipe: MMAs and commits complete in issue order, each at a moment the scheduler
   picks; a commit arrives on its barrier once everything issued before it has completed.
-* TMEM contents as (unit, block) tags: S_t written by an S MMA and read by the softmax
-  warps; P_t written by each softmax warp (its 32 lanes) and read by P.V; O_t, which the
-  softmax rescales between blocks.
+  An MMA reads its shared-memory operands until it completes.
+* TMEM contents as (unit, block) tags: S_t written by an S MMA and loaded by the softmax
+  warps; P_t written by each softmax warp (its 32 lanes) and read by P.V; O_t accumulated
+  by P.V, rescaled by the softmax between blocks and read out by the epilogue.
 * softmax warps, four per tile.  A warp whose 32 rows are all padding skips the loads and
-  the math but keeps every hand-off (one arrival per warp stands for its 32 threads).
-* two schedules: P written over S (the next S_t is issued after P_t.V), and P in columns
-  of its own (the next block's S_t is issued once every warp has read S_t, before P_t.V).
+  the math but keeps every hand-off (one arrival per warp stands for its 32 threads; the
+  epilogue's arrival stands for its warpgroup's).
+* the two MMA schedules of the kernel:
+  - P over S (d = 128 and e4m3): per block, P_t.V then the next S_t, tile by tile; a tile
+    that finishes its unit issues the next unit's first S_t at once, when the ring entry
+    that K_0 of that unit replaces was released by an earlier iteration (the ring-position
+    rule);
+  - P in columns of its own (d = 64, bf16): per block, the next S_t of every tile once its
+    softmax has loaded S_t ("S read"), then P_t.V of every tile, each committed to
+    "P.V done".
 
-Not modelled: TMA loads and the K/V ring, the Q buffers and the epilogue; they have
-barriers of their own and the GPU tests cover them.
+Not modelled: the row statistics the softmax posts for the epilogue, and the arithmetic.
 
 Test infrastructure only: nothing here is used by the library.
 """
@@ -54,98 +65,253 @@ TILES = 2
 
 
 class Cta:
-    """units: per unit, the key blocks of each tile, e.g. [(3, 4), (0, 2)].
+    """units: per unit of this CTA, the key blocks of each tile, e.g. [(3, 4), (0, 2)].
     idle: per unit, per tile, the set of warps whose rows are all padding.
     separate_p: P in columns of its own (else P over S).
-    drop: waits to leave out, for planting a mistake: "s_free" (the MMA warp's wait before
-    the next S), "p_free" (a softmax warp's wait before writing P and O), "idle_p_free" (a
-    padding-only warp's wait before it arrives on p_full); separate P only."""
+    slots: K/V ring slots (the kernel has 4 at d = 128 and 8 at d = 64).
+    drop: waits to leave out, for planting a mistake:
+      "s_free"      the MMA warp's wait for "S read" before the next S (separate P);
+      "p_free"      a softmax warp's wait for the previous P.V before writing P and O
+                    (separate P);
+      "idle_p_free" a padding-only warp's wait for the previous P.V before it arrives on
+                    "P ready" (separate P);
+      "ring_rule"   the ring-position condition on the early first S (P over S);
+      "o_empty"     the MMA warp's wait for the epilogue before a unit's first P.V;
+      "kv_empty"    the producer's wait for a free ring slot;
+      "q_empty"     the producer's wait before it reloads a Q buffer."""
 
-    WAITS = ("s_free", "p_free", "idle_p_free")
+    WAITS = ("s_free", "p_free", "idle_p_free", "ring_rule", "o_empty", "kv_empty", "q_empty")
 
-    def __init__(self, units, idle, separate_p=True, drop=()):
+    def __init__(self, units, idle, separate_p=True, slots=None, drop=()):
         assert set(drop) <= set(self.WAITS)
         self.units, self.idle = units, idle
         self.sep, self.drop = separate_p, set(drop)
+        self.slots = slots or (8 if separate_p else 4)
+        B = Barrier
         self.bars = {}
+        for s in range(self.slots):
+            self.bars["kv_full", s] = B(f"kv_full{s}", 1)
+            self.bars["kv_empty", s] = B(f"kv_empty{s}", 1)
         for t in range(TILES):
-            self.bars["s_full", t] = Barrier(f"s_full{t}", 1)
-            self.bars["p_full", t] = Barrier(f"p_full{t}", WARPS)
-            if separate_p:
-                self.bars["s_free", t] = Barrier(f"s_free{t}", WARPS)
-                self.bars["p_free", t] = Barrier(f"p_free{t}", 1)
+            for name, count in (("q_full", 1), ("q_empty", 1), ("s_full", 1),
+                                ("p_full", WARPS), ("o_full", 1), ("o_empty", 1),
+                                ("s_free", WARPS), ("p_free", 1)):
+                self.bars[name, t] = B(f"{name}{t}", count)
+        self.kv = [None] * self.slots          # ring slot contents
+        self.kv_readers = [0] * self.slots     # MMAs in flight reading the slot
+        self.q = [None] * TILES
+        self.q_readers = [0] * TILES
         self.S = [None] * TILES
         self.P = [[None] * WARPS for _ in range(TILES)]
         self.s_unread = [set() for _ in range(TILES)]  # warps yet to load the current S_t
+        self.O = [None] * TILES                # (unit, blocks accumulated)
+        self.o_read = [True] * TILES           # the epilogue has read the last unit's O_t
         self.pv_in_flight = [0] * TILES
-        self.pipe = []
+        self.pipe = []                         # tensor pipe, in issue order
+        self.tma = []                          # loads in flight, any completion order
         self.pv_done = []
+        self.epilogue_done = []
 
-    # ---------------------------------------------------------------- tensor pipe
+    # ---------------------------------------------------------------- async engines
     def issue(self, op):
-        if op[0] == "PV":
+        if op[0] == "S":
+            self.kv_readers[op[2]] += 1
+            self.q_readers[op[1]] += 1
+        elif op[0] == "PV":
+            self.kv_readers[op[2]] += 1
             self.pv_in_flight[op[1]] += 1
         self.pipe.append(op)
 
-    def complete_one(self):
+    def complete_mma(self):
         op = self.pipe.pop(0)
         if op[0] == "S":
-            _, t, tag = op
+            _, t, slot, (u, it) = op
+            if self.kv[slot] != ("K", u, it) or self.q[t] != u:
+                raise Race(f"S_{t} of {(u, it)} read K {self.kv[slot]} and Q of unit {self.q[t]}")
+            self.kv_readers[slot] -= 1
+            self.q_readers[t] -= 1
             if self.s_unread[t]:
-                raise Race(f"S_{t} of {tag} written before warps {sorted(self.s_unread[t])} "
+                raise Race(f"S_{t} of {(u, it)} written before warps {sorted(self.s_unread[t])} "
                            f"loaded S of {self.S[t]}")
-            self.S[t] = tag
-            self.s_unread[t] = set(range(WARPS)) - self.idle[tag[0]][t]
+            self.S[t] = (u, it)
+            self.s_unread[t] = set(range(WARPS)) - self.idle[u][t]
             if not self.sep:
                 self.P[t] = [None] * WARPS  # P lives in S's columns
         elif op[0] == "PV":
-            _, t, tag = op
+            _, t, slot, (u, it) = op
+            if self.kv[slot] != ("V", u, it):
+                raise Race(f"P_{t}.V of {(u, it)} read V {self.kv[slot]}")
             for w in range(WARPS):
-                if w not in self.idle[tag[0]][t] and self.P[t][w] != tag:
-                    raise Race(f"P_{t}.V of {tag} read warp {w}'s P of {self.P[t][w]}")
+                if w not in self.idle[u][t] and self.P[t][w] != (u, it):
+                    raise Race(f"P_{t}.V of {(u, it)} read warp {w}'s P of {self.P[t][w]}")
+            if it == 0:
+                if not self.o_read[t]:
+                    raise Race(f"P_{t}.V of {(u, it)} overwrote O of {self.O[t]} before the epilogue read it")
+                self.o_read[t] = False
+            elif self.O[t] != (u, it):
+                raise Race(f"P_{t}.V of {(u, it)} accumulated onto O of {self.O[t]}")
+            self.O[t] = (u, it + 1)
+            self.kv_readers[slot] -= 1
             self.pv_in_flight[t] -= 1
-            self.pv_done.append((t, tag))
+            self.pv_done.append((t, (u, it)))
         else:
             self.bars[op[1]].arrive()
 
-    # ---------------------------------------------------------------- MMA warp
+    def complete_tma(self, i):
+        kind, where, tag = self.tma.pop(i)
+        if kind == "Q":
+            if self.q_readers[where]:
+                raise Race(f"Q_{where} of unit {tag} landed while an S MMA read the buffer")
+            self.q[where] = tag
+            self.bars["q_full", where].arrive()
+        else:
+            if self.kv_readers[where]:
+                raise Race(f"{kind} of {tag} landed in slot {where} while an MMA read it")
+            self.kv[where] = (kind,) + tag
+            self.bars["kv_full", where].arrive()
+
     def _wait(self, key, parity):
         bar = self.bars[key]
         return lambda: bar.done(parity)
 
-    def mma(self):
-        pn = [0] * TILES  # p_full waits per tile
-        sf = [0] * TILES  # s_free waits per tile (separate P)
+    # ---------------------------------------------------------------- TMA producer
+    def producer(self):
+        ld, qn = 0, [0] * TILES
+
+        def load_q(u, n, t):
+            if n[t] == 0:
+                return
+            if qn[t] > 0 and "q_empty" not in self.drop:
+                yield self._wait(("q_empty", t), (qn[t] - 1) & 1)
+            self.tma.append(("Q", t, u))
+            qn[t] += 1
+
         for u, n in enumerate(self.units):
+            yield from load_q(u, n, 0)
+            for it in range(max(n)):
+                for kind in ("K", "V"):
+                    slot = ld % self.slots
+                    if ld >= self.slots and "kv_empty" not in self.drop:
+                        yield self._wait(("kv_empty", slot), ((ld // self.slots) - 1) & 1)
+                    self.tma.append((kind, slot, (u, it)))
+                    ld += 1
+                    if it == 0 and kind == "K":
+                        for t in range(1, TILES):
+                            yield from load_q(u, n, t)
+                yield None
+
+    # ---------------------------------------------------------------- MMA warp
+    def mma(self):
+        st = dict(ld=0, qn=[0] * TILES, pn=[0] * TILES, on=[0] * TILES, sf=[0] * TILES)
+        yield from (self._mma_separate_p(st) if self.sep else self._mma_p_over_s(st))
+
+    def _wait_kv(self, st, index):
+        return self._wait(("kv_full", index % self.slots), (index // self.slots) & 1)
+
+    def _issue_s(self, st, t, slot, tag, n_t):
+        """Q_t must have landed; then S_t, its commit, and Q_t's release after the last S_t."""
+        yield self._wait(("q_full", t), st["qn"][t] & 1) if tag[1] == 0 else None
+        if tag[1] == 0:
+            st["qn"][t] += 1
+        self.issue(("S", t, slot, tag))
+        self.issue(("commit", ("s_full", t)))
+        if tag[1] + 1 == n_t:
+            self.issue(("commit", ("q_empty", t)))
+
+    def _issue_pv(self, st, t, slot, tag):
+        yield self._wait(("p_full", t), st["pn"][t] & 1)
+        st["pn"][t] += 1
+        if tag[1] == 0 and st["on"][t] > 0 and "o_empty" not in self.drop:
+            yield self._wait(("o_empty", t), (st["on"][t] - 1) & 1)
+        self.issue(("PV", t, slot, tag))
+
+    def _mma_p_over_s(self, st):
+        early = [False] * TILES
+        for ui, n in enumerate(self.units):
+            n_next = self.units[ui + 1] if ui + 1 < len(self.units) else (0,) * TILES
+            early_next = [False] * TILES
             nblk = max(n)
             if nblk == 0:
                 continue
+            ld_unit = st["ld"]
+            slot_k = st["ld"] % self.slots
+            yield self._wait_kv(st, st["ld"])
+            st["ld"] += 1
+            for t in range(TILES):
+                if n[t] and not early[t]:
+                    yield from self._issue_s(st, t, slot_k, (ui, 0), n[t])
+            self.issue(("commit", ("kv_empty", slot_k)))
+            for it in range(nblk):
+                slot_v = st["ld"] % self.slots
+                yield self._wait_kv(st, st["ld"])
+                st["ld"] += 1
+                nxt = it + 1 < nblk
+                ld_n = st["ld"]
+                slot_n = ld_n % self.slots
+                k_ready = False
+                if nxt:
+                    st["ld"] += 1
+                for t in range(TILES):
+                    if it >= n[t]:
+                        continue
+                    yield from self._issue_pv(st, t, slot_v, (ui, it))
+                    if it + 1 < n[t]:
+                        if not k_ready:
+                            yield self._wait_kv(st, ld_n)
+                            k_ready = True
+                        yield from self._issue_s(st, t, slot_n, (ui, it + 1), n[t])
+                    else:
+                        self.issue(("commit", ("o_full", t)))
+                        st["on"][t] += 1
+                        rule = 2 * (nblk - it) <= self.slots or "ring_rule" in self.drop
+                        if n_next[t] > 0 and rule:
+                            kq = ld_unit + 2 * nblk
+                            yield self._wait_kv(st, kq)
+                            yield from self._issue_s(st, t, kq % self.slots, (ui + 1, 0), n_next[t])
+                            early_next[t] = True
+                    yield None
+                self.issue(("commit", ("kv_empty", slot_v)))
+                if nxt:
+                    self.issue(("commit", ("kv_empty", slot_n)))
+            early = early_next
+
+    def _mma_separate_p(self, st):
+        for ui, n in enumerate(self.units):
+            nblk = max(n)
+            if nblk == 0:
+                continue
+            slot_k = st["ld"] % self.slots
+            yield self._wait_kv(st, st["ld"])
+            st["ld"] += 1
             for t in range(TILES):
                 if n[t]:
-                    self.issue(("S", t, (u, 0)))
-                    self.issue(("commit", ("s_full", t)))
-            yield None
+                    yield from self._issue_s(st, t, slot_k, (ui, 0), n[t])
+            self.issue(("commit", ("kv_empty", slot_k)))
             for it in range(nblk):
-                if self.sep and it + 1 < nblk:
+                slot_v = st["ld"] % self.slots
+                yield self._wait_kv(st, st["ld"])
+                st["ld"] += 1
+                if it + 1 < nblk:
+                    slot_n = st["ld"] % self.slots
+                    yield self._wait_kv(st, st["ld"])
+                    st["ld"] += 1
                     for t in range(TILES):
                         if it + 1 >= n[t]:
                             continue
                         if "s_free" not in self.drop:
-                            yield self._wait(("s_free", t), sf[t] & 1)
-                        sf[t] += 1
-                        self.issue(("S", t, (u, it + 1)))
-                        self.issue(("commit", ("s_full", t)))
+                            yield self._wait(("s_free", t), st["sf"][t] & 1)
+                        st["sf"][t] += 1
+                        yield from self._issue_s(st, t, slot_n, (ui, it + 1), n[t])
+                    self.issue(("commit", ("kv_empty", slot_n)))
                 for t in range(TILES):
                     if it >= n[t]:
                         continue
-                    yield self._wait(("p_full", t), pn[t] & 1)
-                    pn[t] += 1
-                    self.issue(("PV", t, (u, it)))
-                    if self.sep:
-                        self.issue(("commit", ("p_free", t)))
-                    elif it + 1 < n[t]:
-                        self.issue(("S", t, (u, it + 1)))
-                        self.issue(("commit", ("s_full", t)))
+                    yield from self._issue_pv(st, t, slot_v, (ui, it))
+                    self.issue(("commit", ("p_free", t)))
+                    if it + 1 == n[t]:
+                        self.issue(("commit", ("o_full", t)))
+                        st["on"][t] += 1
+                self.issue(("commit", ("kv_empty", slot_v)))
                 yield None
 
     # ---------------------------------------------------------------- softmax warp
@@ -173,53 +339,83 @@ class Cta:
                     continue
                 if self.sep and "p_free" not in self.drop and sn > 1:
                     yield self._wait(("p_free", t), sn & 1)
-                # O rescale and P stores: the previous P.V must be complete
+                # P stores, and (past the first block) the O rescale: the previous P.V must
+                # be complete
                 if self.pv_in_flight[t]:
-                    raise Race(f"softmax {t}.{w} wrote P/O of {(u, it)} while P.V in flight")
+                    raise Race(f"softmax {t}.{w} wrote P of {(u, it)} while P.V was in flight")
+                if it > 0 and self.O[t] != (u, it):
+                    raise Race(f"softmax {t}.{w} rescaled O of {self.O[t]} at block {(u, it)}")
                 self.P[t][w] = (u, it)
                 yield None
                 self.bars["p_full", t].arrive()
 
+    # ---------------------------------------------------------------- epilogue
+    def epilogue(self):
+        oe = [0] * TILES
+        for u, n in enumerate(self.units):
+            for t in range(TILES):
+                if n[t] == 0:
+                    continue
+                yield self._wait(("o_full", t), oe[t] & 1)
+                oe[t] += 1
+                if self.O[t] != (u, n[t]):
+                    raise Race(f"epilogue read O_{t} of {self.O[t]} for unit {u}")
+                yield None
+                if self.O[t] != (u, n[t]):
+                    raise Race(f"O_{t} of unit {u} changed while the epilogue read it")
+                self.o_read[t] = True
+                self.epilogue_done.append((t, u))
+                self.bars["o_empty", t].arrive()
+
     # ---------------------------------------------------------------- scheduler
-    def run(self, rng, max_steps=200000):
-        """Interleave the actors at random (each with a random speed) until all finish."""
-        actors = [self.mma()] + [self.softmax(t, w) for t in range(TILES) for w in range(WARPS)]
-        speed = [rng.uniform(0.02, 1.0) for _ in range(len(actors) + 1)]  # last: the pipe
-        cond = [None] * len(actors)
-        live = list(range(len(actors)))
+    def run(self, rng, max_steps=400000):
+        """Interleave the actors and the two async engines at random, each with a random
+        speed, until everything has finished."""
+        actors = [self.producer(), self.mma(), self.epilogue()] + \
+            [self.softmax(t, w) for t in range(TILES) for w in range(WARPS)]
+        na = len(actors)
+        speed = [rng.uniform(0.02, 1.0) for _ in range(na + 2)]  # + tensor pipe, TMA
+        cond = [None] * na
+        live = list(range(na))
         for _ in range(max_steps):
             runnable = [i for i in live if cond[i] is None or cond[i]()]
             if self.pipe:
-                runnable.append(len(actors))
+                runnable.append(na)
+            if self.tma:
+                runnable.append(na + 1)
             if not runnable:
                 if live:
-                    raise Deadlock(f"{len(live)} actors blocked, pipe empty")
+                    raise Deadlock(f"{len(live)} actors blocked with nothing in flight")
                 break
             i = rng.choices(runnable, weights=[speed[j] for j in runnable])[0]
-            if i == len(actors):
-                self.complete_one()
-                continue
-            try:
-                cond[i] = next(actors[i])
-            except StopIteration:
-                live.remove(i)
+            if i == na:
+                self.complete_mma()
+            elif i == na + 1:
+                self.complete_tma(rng.randrange(len(self.tma)))
+            else:
+                try:
+                    cond[i] = next(actors[i])
+                except StopIteration:
+                    live.remove(i)
         else:
             raise Deadlock("step limit")
         want = sorted((t, (u, it)) for u, n in enumerate(self.units)
                       for t in range(TILES) for it in range(n[t]))
         if sorted(self.pv_done) != want:
             raise Race("not every block's P.V completed")
+        if sorted(self.epilogue_done) != sorted((t, u) for u, n in enumerate(self.units)
+                                                for t in range(TILES) if n[t]):
+            raise Race("not every tile's output was read out")
 
 
-def random_cta(rng, separate_p=True, drop=()):
-    """One to four units per CTA, 0-4 key blocks per tile, random padding-only warps (warp 0
+def random_cta(rng, separate_p=True, slots=None, drop=()):
+    """One to five units per CTA, 0-4 key blocks per tile, random padding-only warps (warp 0
     of a tile with keys always holds a valid row)."""
     units, idle = [], []
-    for _ in range(rng.randint(1, 4)):
-        n = (rng.randint(0, 4), rng.randint(0, 4))
-        units.append(n)
+    for _ in range(rng.randint(1, 5)):
+        units.append((rng.randint(0, 4), rng.randint(0, 4)))
         idle.append([set(w for w in (1, 2, 3) if rng.random() < 0.5) for _ in range(TILES)])
-    return Cta(units, idle, separate_p, drop)
+    return Cta(units, idle, separate_p, slots, drop)
 
 
 def run_random(seed, **kw):

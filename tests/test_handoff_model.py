@@ -1,20 +1,41 @@
-"""The two-tile kernel's MMA / softmax hand-off protocol, checked on a CPU model under random
-interleavings (tests/handoff_model.py).
+"""The two-tile kernel's barrier protocol (TMA producer, MMA warp, softmax warps, epilogue),
+checked on a CPU model under random interleavings (tests/handoff_model.py).
 
 * The model's barrier follows the PTX parity rule, including the aliasing of a waiter two
   phases behind.
-* Both schedules of the kernel, P over S (d = 128, e4m3) and P in columns of its own
-  (d = 64 bf16), finish every block with every consumer seeing the right block's data,
-  with padding-only warps anywhere but warp 0 and units of unequal, possibly empty, tiles.
-* Leaving out any one wait of the separate-P schedule is caught.  Leaving out the
-  padding-only warps' wait reproduces what a B200 showed for an earlier build: P.V ran on
-  a P still holding an older block, while the statistics (and so the LSE) stayed right.
+* Both MMA schedules of the kernel, P over S (d = 128, e4m3) and P in columns of its own
+  (d = 64, bf16), finish every block, and every consumer sees the right block's data.
+  That holds for TMA copies landing in any order, padding-only warps anywhere but warp 0,
+  and several units of unequal, possibly empty, tiles per CTA.
+* Leaving out any one wait is caught, as a wrong read, an overwrite in use or a deadlock.
+  - Leaving out the padding-only warps' wait reproduces what a B200 showed for an earlier
+    build: P.V ran on a P still holding an older block, while the row statistics (and so
+    the LSE) stayed right.
+  - Leaving out the ring-position rule of P over S's early first S deadlocks: K_0 of the
+    next unit would wait for a ring slot this unit has not released yet.
 """
+import random
+
 import pytest
 
 from tests import handoff_model as H
 
 SEEDS = range(400)
+SCHEDULES = {"separate P": True, "P over S": False}
+ONLY_SEPARATE_P = {"s_free", "p_free", "idle_p_free"}
+ONLY_P_OVER_S = {"ring_rule"}
+
+
+def outcomes(separate_p, drop=()):
+    races, deadlocks = [], []
+    for seed in SEEDS:
+        try:
+            H.run_random(seed, separate_p=separate_p, drop=drop)
+        except H.Race as e:
+            races.append(str(e))
+        except H.Deadlock as e:
+            deadlocks.append(str(e))
+    return races, deadlocks
 
 
 def test_barrier_follows_the_parity_rule():
@@ -30,41 +51,40 @@ def test_barrier_follows_the_parity_rule():
     assert not b.done(0) and b.done(1)
 
 
-@pytest.mark.parametrize("separate_p", [True, False], ids=["separate P", "P over S"])
-def test_schedule_is_race_free(separate_p):
-    for seed in SEEDS:
-        H.run_random(seed, separate_p=separate_p)
-
-
-def test_model_covers_the_kernel_geometry():
-    # the random CTAs include empty tiles, unequal tiles, several units and idle warps
-    seen = dict(empty=False, unequal=False, units=False, idle=False)
-    import random
+def test_random_ctas_cover_the_kernel_geometry():
+    seen = dict(empty_tile=False, unequal_tiles=False, units=False, idle=False, empty_unit=False)
     for seed in SEEDS:
         c = H.random_cta(random.Random(seed))
-        seen["empty"] |= any(0 in n and max(n) > 0 for n in c.units)
-        seen["unequal"] |= any(n[0] != n[1] and min(n) > 0 for n in c.units)
-        seen["units"] |= len(c.units) >= 3
+        seen["empty_tile"] |= any(0 in n and max(n) > 0 for n in c.units)
+        seen["unequal_tiles"] |= any(n[0] != n[1] and min(n) > 0 for n in c.units)
+        seen["units"] |= len(c.units) >= 4
         seen["idle"] |= any(any(s) for s in c.idle)
+        seen["empty_unit"] |= any(max(n) == 0 for n in c.units)
     assert all(seen.values()), seen
 
 
-@pytest.mark.parametrize("wait", H.Cta.WAITS)
-def test_every_wait_of_the_separate_p_schedule_is_needed(wait):
-    failures = 0
-    for seed in SEEDS:
-        try:
-            H.run_random(seed, drop=(wait,))
-        except (H.Race, H.Deadlock):
-            failures += 1
-    assert failures > 0, f"leaving out {wait} went unnoticed"
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_schedule_is_race_and_deadlock_free(schedule):
+    races, deadlocks = outcomes(SCHEDULES[schedule])
+    assert not races and not deadlocks, (races[:3], deadlocks[:3])
+
+
+CASES = [(s, w) for s in SCHEDULES for w in H.Cta.WAITS
+         if not (SCHEDULES[s] and w in ONLY_P_OVER_S)
+         and not (not SCHEDULES[s] and w in ONLY_SEPARATE_P)]
+
+
+@pytest.mark.parametrize("schedule,wait", CASES, ids=[f"{s}-{w}" for s, w in CASES])
+def test_every_wait_is_needed(schedule, wait):
+    races, deadlocks = outcomes(SCHEDULES[schedule], drop=(wait,))
+    assert races or deadlocks, f"leaving out {wait} went unnoticed"
 
 
 def test_idle_warp_race_reads_an_older_p():
-    symptoms = []
-    for seed in SEEDS:
-        try:
-            H.run_random(seed, drop=("idle_p_free",))
-        except H.Race as e:
-            symptoms.append(str(e))
-    assert any(".V of" in s and "read warp" in s for s in symptoms), symptoms[:5]
+    races, _ = outcomes(True, drop=("idle_p_free",))
+    assert any(".V of" in r and "read warp" in r for r in races), races[:5]
+
+
+def test_ring_rule_prevents_a_deadlock():
+    races, deadlocks = outcomes(False, drop=("ring_rule",))
+    assert deadlocks and not races, (races[:3], deadlocks[:3])
