@@ -35,6 +35,32 @@ STATUS_NAMES = {
 GQA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
+def _nvtx_enabled() -> bool:
+    return os.environ.get("GQA_NVTX", "") not in ("", "0")
+
+
+class _range:
+    """An NVTX range named after the entry point around each library call, when GQA_NVTX is
+    set (for timeline profilers); otherwise nothing.  It marks the host-side call, inside
+    which the kernels are launched."""
+
+    def __init__(self, name: str):
+        self.name = name
+        self.on = _nvtx_enabled()
+
+    def __enter__(self):
+        if self.on:
+            import torch
+            torch.cuda.nvtx.range_push(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        if self.on:
+            import torch
+            torch.cuda.nvtx.range_pop()
+        return False
+
+
 class GqaError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
@@ -146,7 +172,7 @@ def gqa_attn_fwd(q, k, v, out=None, lse=None, scale=None, causal=False, pack_gqa
         scale = 1.0 / math.sqrt(d)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    with torch.cuda.device(q.device):
+    with torch.cuda.device(q.device), _range(_entry):
         _check(getattr(load(), _entry)(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                        out.data_ptr(), lse.data_ptr(), B, Sq, Sk, Hq, Hk, d,
                                        float(scale), int(bool(causal)), int(pack_gqa),
@@ -211,7 +237,7 @@ def gqa_attn_fwd_kvcache(q, k_cache, v_cache, cache_seqlens=None, out=None, lse=
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     code = GQA_OUT_BF16 if out.dtype == torch.bfloat16 else GQA_OUT_F32
-    with torch.cuda.device(q.device):
+    with torch.cuda.device(q.device), _range("gqa_attn_fwd_kvcache"):
         _check(load().gqa_attn_fwd_kvcache(
             q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
             None if cache_seqlens is None else cache_seqlens.data_ptr(), out.data_ptr(), code,
@@ -260,7 +286,7 @@ def gqa_attn_fwd_paged(q, k_pages, v_pages, block_table, cache_seqlens, out=None
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     code = GQA_OUT_BF16 if out.dtype == torch.bfloat16 else GQA_OUT_F32
-    with torch.cuda.device(q.device):
+    with torch.cuda.device(q.device), _range("gqa_attn_fwd_paged"):
         _check(load().gqa_attn_fwd_paged(
             q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
             int(block_table.shape[1]), cache_seqlens.data_ptr(), num_pages, page_size,
@@ -308,7 +334,7 @@ def gqa_attn_fwd_fp8(q, k, v, q_scale, k_scale, v_scale, cache_seqlens=None, out
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     code = GQA_OUT_BF16 if out.dtype == torch.bfloat16 else GQA_OUT_F32
-    with torch.cuda.device(q.device):
+    with torch.cuda.device(q.device), _range("gqa_attn_fwd_fp8"):
         _check(load().gqa_attn_fwd_fp8(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), float(q_scale), float(k_scale),
             float(v_scale), None if cache_seqlens is None else cache_seqlens.data_ptr(),

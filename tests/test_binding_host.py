@@ -35,3 +35,22 @@ def test_kvcache_refuses_mismatched_cache_shapes():
     q = _cpu((2, 1, 4, 64))
     with pytest.raises(ValueError):
         G.gqa_attn_fwd_kvcache(q, _cpu((2, 16, 2, 64)), _cpu((2, 8, 2, 64)))
+
+
+def test_nvtx_ranges_only_when_asked(monkeypatch):
+    calls = []
+    monkeypatch.setattr(torch.cuda.nvtx, "range_push", lambda name: calls.append(("push", name)))
+    monkeypatch.setattr(torch.cuda.nvtx, "range_pop", lambda: calls.append(("pop",)))
+    monkeypatch.delenv("GQA_NVTX", raising=False)
+    with G._range("gqa_attn_fwd"):
+        pass
+    assert calls == []
+    monkeypatch.setenv("GQA_NVTX", "0")
+    with G._range("gqa_attn_fwd"):
+        pass
+    assert calls == []
+    monkeypatch.setenv("GQA_NVTX", "1")
+    with pytest.raises(RuntimeError):
+        with G._range("gqa_attn_fwd_paged"):
+            raise RuntimeError("a failed call still closes its range")
+    assert calls == [("push", "gqa_attn_fwd_paged"), ("pop",)]
