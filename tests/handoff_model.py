@@ -1,6 +1,7 @@
-"""A discrete-event model of one CTA of the two-tile forward kernel, for checking its barrier
-protocol on the CPU: the TMA producer, the MMA warp, four softmax warps per tile and the
-epilogue, with the hand-offs between them.
+"""A discrete-event model of one CTA of the forward kernel, for checking its barrier protocol
+on the CPU: the TMA producer, the MMA warp, four softmax warps per tile and the epilogue,
+with the hand-offs between them.  Two tiles per CTA (prefill) or one (decode and short
+query axes, where the softmax warps write their own output and release O).
 
 What it models, in the kernel's terms:
 
@@ -61,14 +62,16 @@ class Barrier:
 
 
 WARPS = 4
-TILES = 2
 
 
 class Cta:
     """units: per unit of this CTA, the key blocks of each tile, e.g. [(3, 4), (0, 2)].
     idle: per unit, per tile, the set of warps whose rows are all padding.
-    separate_p: P in columns of its own (else P over S).
-    slots: K/V ring slots (the kernel has 4 at d = 128 and 8 at d = 64).
+    separate_p: P in columns of its own (else P over S; the kernel uses separate P with two
+    bf16 tiles at d = 64 only).
+    slots: K/V ring slots (the kernel has 4 at d = 128 and 8 at d = 64 with two tiles, 2 and
+    5 with one).
+    tiles: 2, with an epilogue warpgroup; or 1, whose softmax warps write the output.
     drop: waits to leave out, for planting a mistake:
       "s_free"      the MMA warp's wait for "S read" before the next S (separate P);
       "p_free"      a softmax warp's wait for the previous P.V before writing P and O
@@ -82,35 +85,38 @@ class Cta:
 
     WAITS = ("s_free", "p_free", "idle_p_free", "ring_rule", "o_empty", "kv_empty", "q_empty")
 
-    def __init__(self, units, idle, separate_p=True, slots=None, drop=()):
-        assert set(drop) <= set(self.WAITS)
+    def __init__(self, units, idle, separate_p=True, slots=None, drop=(), tiles=2):
+        assert set(drop) <= set(self.WAITS) and tiles in (1, 2)
+        assert all(len(n) == tiles for n in units)
         self.units, self.idle = units, idle
-        self.sep, self.drop = separate_p, set(drop)
-        self.slots = slots or (8 if separate_p else 4)
+        self.sep, self.drop, self.nt = separate_p, set(drop), tiles
+        self.slots = slots or ((8 if separate_p else 4) if tiles == 2 else 2)
         B = Barrier
         self.bars = {}
         for s in range(self.slots):
             self.bars["kv_full", s] = B(f"kv_full{s}", 1)
             self.bars["kv_empty", s] = B(f"kv_empty{s}", 1)
-        for t in range(TILES):
+        o_empty_count = 1 if tiles == 2 else WARPS  # the epilogue, or every softmax warp
+        for t in range(tiles):
             for name, count in (("q_full", 1), ("q_empty", 1), ("s_full", 1),
-                                ("p_full", WARPS), ("o_full", 1), ("o_empty", 1),
+                                ("p_full", WARPS), ("o_full", 1), ("o_empty", o_empty_count),
                                 ("s_free", WARPS), ("p_free", 1)):
                 self.bars[name, t] = B(f"{name}{t}", count)
         self.kv = [None] * self.slots          # ring slot contents
         self.kv_readers = [0] * self.slots     # MMAs in flight reading the slot
-        self.q = [None] * TILES
-        self.q_readers = [0] * TILES
-        self.S = [None] * TILES
-        self.P = [[None] * WARPS for _ in range(TILES)]
-        self.s_unread = [set() for _ in range(TILES)]  # warps yet to load the current S_t
-        self.O = [None] * TILES                # (unit, blocks accumulated)
-        self.o_read = [True] * TILES           # the epilogue has read the last unit's O_t
-        self.pv_in_flight = [0] * TILES
+        self.q = [None] * self.nt
+        self.q_readers = [0] * self.nt
+        self.S = [None] * self.nt
+        self.P = [[None] * WARPS for _ in range(self.nt)]
+        self.s_unread = [set() for _ in range(self.nt)]  # warps yet to load the current S_t
+        self.O = [None] * self.nt                # (unit, blocks accumulated)
+        self.o_read = [True] * self.nt           # the epilogue has read the last unit's O_t
+        self.pv_in_flight = [0] * self.nt
         self.pipe = []                         # tensor pipe, in issue order
         self.tma = []                          # loads in flight, any completion order
         self.pv_done = []
         self.epilogue_done = []
+        self.o_readers = 0                     # readers of the current O done (one tile)
 
     # ---------------------------------------------------------------- async engines
     def issue(self, op):
@@ -176,7 +182,7 @@ class Cta:
 
     # ---------------------------------------------------------------- TMA producer
     def producer(self):
-        ld, qn = 0, [0] * TILES
+        ld, qn = 0, [0] * self.nt
 
         def load_q(u, n, t):
             if n[t] == 0:
@@ -196,13 +202,13 @@ class Cta:
                     self.tma.append((kind, slot, (u, it)))
                     ld += 1
                     if it == 0 and kind == "K":
-                        for t in range(1, TILES):
+                        for t in range(1, self.nt):
                             yield from load_q(u, n, t)
                 yield None
 
     # ---------------------------------------------------------------- MMA warp
     def mma(self):
-        st = dict(ld=0, qn=[0] * TILES, pn=[0] * TILES, on=[0] * TILES, sf=[0] * TILES)
+        st = dict(ld=0, qn=[0] * self.nt, pn=[0] * self.nt, on=[0] * self.nt, sf=[0] * self.nt)
         yield from (self._mma_separate_p(st) if self.sep else self._mma_p_over_s(st))
 
     def _wait_kv(self, st, index):
@@ -226,10 +232,10 @@ class Cta:
         self.issue(("PV", t, slot, tag))
 
     def _mma_p_over_s(self, st):
-        early = [False] * TILES
+        early = [False] * self.nt
         for ui, n in enumerate(self.units):
-            n_next = self.units[ui + 1] if ui + 1 < len(self.units) else (0,) * TILES
-            early_next = [False] * TILES
+            n_next = self.units[ui + 1] if ui + 1 < len(self.units) else (0,) * self.nt
+            early_next = [False] * self.nt
             nblk = max(n)
             if nblk == 0:
                 continue
@@ -237,7 +243,7 @@ class Cta:
             slot_k = st["ld"] % self.slots
             yield self._wait_kv(st, st["ld"])
             st["ld"] += 1
-            for t in range(TILES):
+            for t in range(self.nt):
                 if n[t] and not early[t]:
                     yield from self._issue_s(st, t, slot_k, (ui, 0), n[t])
             self.issue(("commit", ("kv_empty", slot_k)))
@@ -251,7 +257,7 @@ class Cta:
                 k_ready = False
                 if nxt:
                     st["ld"] += 1
-                for t in range(TILES):
+                for t in range(self.nt):
                     if it >= n[t]:
                         continue
                     yield from self._issue_pv(st, t, slot_v, (ui, it))
@@ -283,7 +289,7 @@ class Cta:
             slot_k = st["ld"] % self.slots
             yield self._wait_kv(st, st["ld"])
             st["ld"] += 1
-            for t in range(TILES):
+            for t in range(self.nt):
                 if n[t]:
                     yield from self._issue_s(st, t, slot_k, (ui, 0), n[t])
             self.issue(("commit", ("kv_empty", slot_k)))
@@ -295,7 +301,7 @@ class Cta:
                     slot_n = st["ld"] % self.slots
                     yield self._wait_kv(st, st["ld"])
                     st["ld"] += 1
-                    for t in range(TILES):
+                    for t in range(self.nt):
                         if it + 1 >= n[t]:
                             continue
                         if "s_free" not in self.drop:
@@ -303,7 +309,7 @@ class Cta:
                         st["sf"][t] += 1
                         yield from self._issue_s(st, t, slot_n, (ui, it + 1), n[t])
                     self.issue(("commit", ("kv_empty", slot_n)))
-                for t in range(TILES):
+                for t in range(self.nt):
                     if it >= n[t]:
                         continue
                     yield from self._issue_pv(st, t, slot_v, (ui, it))
@@ -317,6 +323,7 @@ class Cta:
     # ---------------------------------------------------------------- softmax warp
     def softmax(self, t, w):
         sn = 0  # S blocks of this tile so far
+        so = 0  # outputs of this tile written (one tile per CTA)
         for u, n in enumerate(self.units):
             nt = n[t]
             if nt == 0:
@@ -348,31 +355,44 @@ class Cta:
                 self.P[t][w] = (u, it)
                 yield None
                 self.bars["p_full", t].arrive()
+            if self.nt == 1:
+                # one tile per CTA: every warp (padding-only ones too) waits for the finished
+                # O, writes its rows out and releases them
+                yield self._wait(("o_full", t), so & 1)
+                so += 1
+                yield from self._read_out(t, u, nt, f"softmax {t}.{w}")
+                self.bars["o_empty", t].arrive()
+
+    def _read_out(self, t, u, n_t, who):
+        if self.O[t] != (u, n_t):
+            raise Race(f"{who} read O_{t} of {self.O[t]} for unit {u}")
+        yield None
+        if self.O[t] != (u, n_t):
+            raise Race(f"O_{t} of unit {u} changed while {who} read it")
+        self.o_readers += 1
+        if self.o_readers == self.bars["o_empty", t].count:
+            self.o_readers = 0
+            self.o_read[t] = True
+            self.epilogue_done.append((t, u))
 
     # ---------------------------------------------------------------- epilogue
     def epilogue(self):
-        oe = [0] * TILES
+        oe = [0] * self.nt
         for u, n in enumerate(self.units):
-            for t in range(TILES):
+            for t in range(self.nt):
                 if n[t] == 0:
                     continue
                 yield self._wait(("o_full", t), oe[t] & 1)
                 oe[t] += 1
-                if self.O[t] != (u, n[t]):
-                    raise Race(f"epilogue read O_{t} of {self.O[t]} for unit {u}")
-                yield None
-                if self.O[t] != (u, n[t]):
-                    raise Race(f"O_{t} of unit {u} changed while the epilogue read it")
-                self.o_read[t] = True
-                self.epilogue_done.append((t, u))
+                yield from self._read_out(t, u, n[t], "the epilogue")
                 self.bars["o_empty", t].arrive()
 
     # ---------------------------------------------------------------- scheduler
     def run(self, rng, max_steps=400000):
         """Interleave the actors and the two async engines at random, each with a random
         speed, until everything has finished."""
-        actors = [self.producer(), self.mma(), self.epilogue()] + \
-            [self.softmax(t, w) for t in range(TILES) for w in range(WARPS)]
+        actors = [self.producer(), self.mma()] + ([self.epilogue()] if self.nt == 2 else []) + \
+            [self.softmax(t, w) for t in range(self.nt) for w in range(WARPS)]
         na = len(actors)
         speed = [rng.uniform(0.02, 1.0) for _ in range(na + 2)]  # + tensor pipe, TMA
         cond = [None] * na
@@ -400,22 +420,22 @@ class Cta:
         else:
             raise Deadlock("step limit")
         want = sorted((t, (u, it)) for u, n in enumerate(self.units)
-                      for t in range(TILES) for it in range(n[t]))
+                      for t in range(self.nt) for it in range(n[t]))
         if sorted(self.pv_done) != want:
             raise Race("not every block's P.V completed")
         if sorted(self.epilogue_done) != sorted((t, u) for u, n in enumerate(self.units)
-                                                for t in range(TILES) if n[t]):
+                                                for t in range(self.nt) if n[t]):
             raise Race("not every tile's output was read out")
 
 
-def random_cta(rng, separate_p=True, slots=None, drop=()):
+def random_cta(rng, separate_p=True, slots=None, drop=(), tiles=2):
     """One to five units per CTA, 0-4 key blocks per tile, random padding-only warps (warp 0
     of a tile with keys always holds a valid row)."""
     units, idle = [], []
     for _ in range(rng.randint(1, 5)):
-        units.append((rng.randint(0, 4), rng.randint(0, 4)))
-        idle.append([set(w for w in (1, 2, 3) if rng.random() < 0.5) for _ in range(TILES)])
-    return Cta(units, idle, separate_p, slots, drop)
+        units.append(tuple(rng.randint(0, 4) for _ in range(tiles)))
+        idle.append([set(w for w in (1, 2, 3) if rng.random() < 0.5) for _ in range(tiles)])
+    return Cta(units, idle, separate_p, slots, drop, tiles)
 
 
 def run_random(seed, **kw):

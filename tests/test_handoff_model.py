@@ -1,10 +1,13 @@
-"""The two-tile kernel's barrier protocol (TMA producer, MMA warp, softmax warps, epilogue),
+"""The forward kernel's barrier protocol (TMA producer, MMA warp, softmax warps, epilogue),
 checked on a CPU model under random interleavings (tests/handoff_model.py).
 
 * The model's barrier follows the PTX parity rule, including the aliasing of a waiter two
   phases behind.
-* Both MMA schedules of the kernel, P over S (d = 128, e4m3) and P in columns of its own
-  (d = 64, bf16), finish every block, and every consumer sees the right block's data.
+* The kernel's three configurations finish every block, and every consumer sees the right
+  block's data:
+  - two tiles with P over S (d = 128, e4m3);
+  - two tiles with P in columns of its own (d = 64, bf16);
+  - one tile with P over S (decode and short query axes).
   That holds for TMA copies landing in any order, padding-only warps anywhere but warp 0,
   and several units of unequal, possibly empty, tiles per CTA.
 * Leaving out any one wait is caught, as a wrong read, an overwrite in use or a deadlock.
@@ -13,6 +16,10 @@ checked on a CPU model under random interleavings (tests/handoff_model.py).
     the LSE) stayed right.
   - Leaving out the ring-position rule of P over S's early first S deadlocks: K_0 of the
     next unit would wait for a ring slot this unit has not released yet.
+* With one tile, two waits are implied by others, and the model shows it:
+  - the ring-position rule always holds: the tile ends on its unit's last block;
+  - the MMA warp's wait for the released O: the next unit's first P.V already waits for
+    every warp's P, which each warp writes only after reading the last O out.
 """
 import random
 
@@ -21,16 +28,19 @@ import pytest
 from tests import handoff_model as H
 
 SEEDS = range(400)
-SCHEDULES = {"separate P": True, "P over S": False}
+# name: (separate P, tiles)
+SCHEDULES = {"two tiles, separate P": (True, 2), "two tiles, P over S": (False, 2),
+             "one tile, P over S": (False, 1)}
 ONLY_SEPARATE_P = {"s_free", "p_free", "idle_p_free"}
-ONLY_P_OVER_S = {"ring_rule"}
+IMPLIED_WITH_ONE_TILE = {"ring_rule", "o_empty"}
 
 
-def outcomes(separate_p, drop=()):
+def outcomes(schedule, drop=()):
+    separate_p, tiles = SCHEDULES[schedule]
     races, deadlocks = [], []
     for seed in SEEDS:
         try:
-            H.run_random(seed, separate_p=separate_p, drop=drop)
+            H.run_random(seed, separate_p=separate_p, drop=drop, tiles=tiles)
         except H.Race as e:
             races.append(str(e))
         except H.Deadlock as e:
@@ -54,7 +64,7 @@ def test_barrier_follows_the_parity_rule():
 def test_random_ctas_cover_the_kernel_geometry():
     seen = dict(empty_tile=False, unequal_tiles=False, units=False, idle=False, empty_unit=False)
     for seed in SEEDS:
-        c = H.random_cta(random.Random(seed))
+        c = H.random_cta(random.Random(seed), tiles=2)
         seen["empty_tile"] |= any(0 in n and max(n) > 0 for n in c.units)
         seen["unequal_tiles"] |= any(n[0] != n[1] and min(n) > 0 for n in c.units)
         seen["units"] |= len(c.units) >= 4
@@ -65,26 +75,39 @@ def test_random_ctas_cover_the_kernel_geometry():
 
 @pytest.mark.parametrize("schedule", SCHEDULES)
 def test_schedule_is_race_and_deadlock_free(schedule):
-    races, deadlocks = outcomes(SCHEDULES[schedule])
+    races, deadlocks = outcomes(schedule)
     assert not races and not deadlocks, (races[:3], deadlocks[:3])
 
 
-CASES = [(s, w) for s in SCHEDULES for w in H.Cta.WAITS
-         if not (SCHEDULES[s] and w in ONLY_P_OVER_S)
-         and not (not SCHEDULES[s] and w in ONLY_SEPARATE_P)]
+def applies(schedule, wait):
+    separate_p, tiles = SCHEDULES[schedule]
+    if wait in ONLY_SEPARATE_P:
+        return separate_p
+    if wait == "ring_rule" and separate_p:
+        return False  # the separate-P schedule has no early first S
+    return not (tiles == 1 and wait in IMPLIED_WITH_ONE_TILE)
+
+
+CASES = [(s, w) for s in SCHEDULES for w in H.Cta.WAITS if applies(s, w)]
 
 
 @pytest.mark.parametrize("schedule,wait", CASES, ids=[f"{s}-{w}" for s, w in CASES])
 def test_every_wait_is_needed(schedule, wait):
-    races, deadlocks = outcomes(SCHEDULES[schedule], drop=(wait,))
+    races, deadlocks = outcomes(schedule, drop=(wait,))
     assert races or deadlocks, f"leaving out {wait} went unnoticed"
 
 
+@pytest.mark.parametrize("wait", sorted(IMPLIED_WITH_ONE_TILE))
+def test_waits_implied_with_one_tile(wait):
+    races, deadlocks = outcomes("one tile, P over S", drop=(wait,))
+    assert not races and not deadlocks, (races[:3], deadlocks[:3])
+
+
 def test_idle_warp_race_reads_an_older_p():
-    races, _ = outcomes(True, drop=("idle_p_free",))
+    races, _ = outcomes("two tiles, separate P", drop=("idle_p_free",))
     assert any(".V of" in r and "read warp" in r for r in races), races[:5]
 
 
 def test_ring_rule_prevents_a_deadlock():
-    races, deadlocks = outcomes(False, drop=("ring_rule",))
+    races, deadlocks = outcomes("two tiles, P over S", drop=("ring_rule",))
     assert deadlocks and not races, (races[:3], deadlocks[:3])
