@@ -42,6 +42,16 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 CSRC_DIR = os.path.join(ROOT, "gqa_exact_attention_b200", "csrc")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# nominal (datasheet) peaks of one B200, the second denominator every fraction is given
+# against: dense bf16 tensor throughput and HBM3e bandwidth
+SPEC_PEAKS = {"tensor": 2250.0, "hbm": 8000.0}
+
+
+def with_spec(roof):
+    """Add the nominal peak and the fraction of it beside the measured one."""
+    roof["spec_peak"] = SPEC_PEAKS[roof["bound"]]
+    roof["frac_of_spec"] = roof["achieved"] / roof["spec_peak"]
+    return roof
 
 
 # ----------------------------------------------------------------- work accounting
@@ -321,10 +331,11 @@ def run_decode(args, pg, world, rank, dev, peaks, peak_src):
         "tokens_per_s": round(world * B / (total_ms / args.steps / 1e3), 1),
         "pack_gqa": pack, "num_splits": splits, "l2": c["l2"],
         "gpu_launches": (1 + (1 if splits > 1 else 0)) * args.steps,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "peak_source": f"{peak_src}:hbm_gbs",
-                     "traffic": traffic_for(c["name"], pack, splits), "kernel": "gqa_fwd_kernel"},
+        "roofline": with_spec({"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                               "peak_source": f"{peak_src}:hbm_gbs",
+                               "traffic": traffic_for(c["name"], pack, splits),
+                               "kernel": "gqa_fwd_kernel"}),
     }
     del q, k, v, out, lse
     torch.cuda.empty_cache()
@@ -480,6 +491,7 @@ def run_gpu(args, cfg):
     roof["peak_source"] = f"{peak_src}:" + ("hbm_gbs" if decode_like else pk_key)
     roof["traffic"] = traffic_for(cfg["name"], pack, splits)
     roof["kernel"] = "gqa_fwd_kernel"
+    with_spec(roof)
 
     tokens = B * (Sq if Sq > 1 else 1)
     line = {
@@ -510,9 +522,10 @@ def run_gpu(args, cfg):
             "value": round(sus_val, 3), "unit": unit, "steps": sus_steps,
             "timed_s": round(sus_total / 1e3, 3), "ms_per_step": round(sus_ms, 4),
             "gpu_launches": launches_per_step * sus_steps,
-            "roofline": {"bound": "tensor", "achieved": fl / (sus_ms / 1e3) / 1e12, "peak": pk,
-                         "unit": "TFLOP/s", "frac": fl / (sus_ms / 1e3) / 1e12 / pk,
-                         "peak_source": f"{peak_src}:bf16_tflops_sustained"}}
+            "roofline": with_spec({"bound": "tensor", "achieved": fl / (sus_ms / 1e3) / 1e12,
+                                   "peak": pk, "unit": "TFLOP/s",
+                                   "frac": fl / (sus_ms / 1e3) / 1e12 / pk,
+                                   "peak_source": f"{peak_src}:bf16_tflops_sustained"})}
     if decode is not None:
         line["decode"] = decode
     if rank == 0 and not args.no_cpu_baseline:

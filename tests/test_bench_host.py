@@ -96,3 +96,11 @@ def test_committed_traffic_covers_both_objects_of_the_default_line(bench):
         w = t["workloads"][name]
         assert w["algorithmic_bytes"] == bench.hbm_bytes(*shape)
         assert 0.9 < w["dram_bytes_per_launch"] / w["algorithmic_bytes"] < 1.3
+
+
+def test_every_fraction_is_also_given_against_the_nominal_peaks():
+    import bench
+    t = bench.with_spec({"bound": "tensor", "achieved": 1125.0})
+    h = bench.with_spec({"bound": "hbm", "achieved": 6000.0})
+    assert t["spec_peak"] == 2250.0 and t["frac_of_spec"] == 0.5
+    assert h["spec_peak"] == 8000.0 and h["frac_of_spec"] == 0.75
