@@ -528,7 +528,7 @@ def run_gpu(args, cfg):
                                    "peak_source": f"{peak_src}:bf16_tflops_sustained"})}
     if decode is not None:
         line["decode"] = decode
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, threads, desc = oracle_sample(cfg, args.cpu_budget)
         if decode_like:
             cv = by / (fl / rate) / 1e9
@@ -555,6 +555,10 @@ def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    # torchrun gives every rank OMP_NUM_THREADS=1; here rank 0 works alone, so the oracle
+    # gets the host's cores, as in a single-process run (set before its OpenMP starts)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and os.environ.get("OMP_NUM_THREADS") == "1":
+        os.environ["OMP_NUM_THREADS"] = str(len(os.sched_getaffinity(0)))
     B, Sq, Sk, Hq, Hk, d, causal = (cfg[k] for k in ("B", "Sq", "Sk", "Hq", "Hk", "d", "causal"))
     budget = max(2.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
