@@ -81,21 +81,30 @@ class Cta:
       "ring_rule"   the ring-position condition on the early first S (P over S);
       "o_empty"     the MMA warp's wait for the epilogue before a unit's first P.V;
       "kv_empty"    the producer's wait for a free ring slot;
-      "q_empty"     the producer's wait before it reloads a Q buffer."""
+      "q_empty"     the producer's wait before it reloads a Q buffer;
+      "every_index" (two issuers) an issuer's wait for a ring entry its tile does not read,
+                    before it releases that entry.
+    two_issuers: P over S with one MMA-issuing warp per tile (a design under study, not the
+    kernel's): each walks every ring entry in order and releases each (kv_empty counts
+    both), and a tile's early first S follows the same ring-position rule."""
 
-    WAITS = ("s_free", "p_free", "idle_p_free", "ring_rule", "o_empty", "kv_empty", "q_empty")
+    WAITS = ("s_free", "p_free", "idle_p_free", "ring_rule", "o_empty", "kv_empty", "q_empty",
+             "every_index")
 
-    def __init__(self, units, idle, separate_p=True, slots=None, drop=(), tiles=2):
+    def __init__(self, units, idle, separate_p=True, slots=None, drop=(), tiles=2,
+                 two_issuers=False):
         assert set(drop) <= set(self.WAITS) and tiles in (1, 2)
         assert all(len(n) == tiles for n in units)
+        assert not (two_issuers and (separate_p or tiles != 2))
         self.units, self.idle = units, idle
         self.sep, self.drop, self.nt = separate_p, set(drop), tiles
+        self.two_issuers = two_issuers
         self.slots = slots or ((8 if separate_p else 4) if tiles == 2 else 2)
         B = Barrier
         self.bars = {}
         for s in range(self.slots):
             self.bars["kv_full", s] = B(f"kv_full{s}", 1)
-            self.bars["kv_empty", s] = B(f"kv_empty{s}", 1)
+            self.bars["kv_empty", s] = B(f"kv_empty{s}", 2 if two_issuers else 1)
         o_empty_count = 1 if tiles == 2 else WARPS  # the epilogue, or every softmax warp
         for t in range(tiles):
             for name, count in (("q_full", 1), ("q_empty", 1), ("s_full", 1),
@@ -113,23 +122,40 @@ class Cta:
         self.o_read = [True] * self.nt           # the epilogue has read the last unit's O_t
         self.pv_in_flight = [0] * self.nt
         self.pipe = []                         # tensor pipe, in issue order
+        self.issued, self.n_done = 0, 0        # MMAs issued / completed
+        self.last_op = {}                      # per issuer: number of its latest MMA
+        self.commits = []                      # (MMA number to wait for, barrier)
         self.tma = []                          # loads in flight, any completion order
         self.pv_done = []
         self.epilogue_done = []
         self.o_readers = 0                     # readers of the current O done (one tile)
 
     # ---------------------------------------------------------------- async engines
-    def issue(self, op):
+    def issue(self, op, who=0):
         if op[0] == "S":
             self.kv_readers[op[2]] += 1
             self.q_readers[op[1]] += 1
-        elif op[0] == "PV":
+        else:
             self.kv_readers[op[2]] += 1
             self.pv_in_flight[op[1]] += 1
         self.pipe.append(op)
+        self.issued += 1
+        self.last_op[who] = self.issued  # MMA number k has completed once k <= n_done
+
+    def commit(self, key, who=0):
+        """tcgen05.commit: arrive on the barrier once every MMA this issuer has issued so far
+        has completed (another issuer's MMAs do not count)."""
+        self.commits.append((self.last_op.get(who, 0), key))
+
+    def fire_commit(self, i):
+        self.bars[self.commits.pop(i)[1]].arrive()
+
+    def ready_commits(self):
+        return [i for i, (k, _) in enumerate(self.commits) if k <= self.n_done]
 
     def complete_mma(self):
         op = self.pipe.pop(0)
+        self.n_done += 1
         if op[0] == "S":
             _, t, slot, (u, it) = op
             if self.kv[slot] != ("K", u, it) or self.q[t] != u:
@@ -160,8 +186,6 @@ class Cta:
             self.kv_readers[slot] -= 1
             self.pv_in_flight[t] -= 1
             self.pv_done.append((t, (u, it)))
-        else:
-            self.bars[op[1]].arrive()
 
     def complete_tma(self, i):
         kind, where, tag = self.tma.pop(i)
@@ -214,22 +238,22 @@ class Cta:
     def _wait_kv(self, st, index):
         return self._wait(("kv_full", index % self.slots), (index // self.slots) & 1)
 
-    def _issue_s(self, st, t, slot, tag, n_t):
+    def _issue_s(self, st, t, slot, tag, n_t, who=0):
         """Q_t must have landed; then S_t, its commit, and Q_t's release after the last S_t."""
         yield self._wait(("q_full", t), st["qn"][t] & 1) if tag[1] == 0 else None
         if tag[1] == 0:
             st["qn"][t] += 1
-        self.issue(("S", t, slot, tag))
-        self.issue(("commit", ("s_full", t)))
+        self.issue(("S", t, slot, tag), who)
+        self.commit(("s_full", t), who)
         if tag[1] + 1 == n_t:
-            self.issue(("commit", ("q_empty", t)))
+            self.commit(("q_empty", t), who)
 
-    def _issue_pv(self, st, t, slot, tag):
+    def _issue_pv(self, st, t, slot, tag, who=0):
         yield self._wait(("p_full", t), st["pn"][t] & 1)
         st["pn"][t] += 1
         if tag[1] == 0 and st["on"][t] > 0 and "o_empty" not in self.drop:
             yield self._wait(("o_empty", t), (st["on"][t] - 1) & 1)
-        self.issue(("PV", t, slot, tag))
+        self.issue(("PV", t, slot, tag), who)
 
     def _mma_p_over_s(self, st):
         early = [False] * self.nt
@@ -246,7 +270,7 @@ class Cta:
             for t in range(self.nt):
                 if n[t] and not early[t]:
                     yield from self._issue_s(st, t, slot_k, (ui, 0), n[t])
-            self.issue(("commit", ("kv_empty", slot_k)))
+            self.commit(("kv_empty", slot_k))
             for it in range(nblk):
                 slot_v = st["ld"] % self.slots
                 yield self._wait_kv(st, st["ld"])
@@ -267,7 +291,7 @@ class Cta:
                             k_ready = True
                         yield from self._issue_s(st, t, slot_n, (ui, it + 1), n[t])
                     else:
-                        self.issue(("commit", ("o_full", t)))
+                        self.commit(("o_full", t))
                         st["on"][t] += 1
                         rule = 2 * (nblk - it) <= self.slots or "ring_rule" in self.drop
                         if n_next[t] > 0 and rule:
@@ -276,9 +300,63 @@ class Cta:
                             yield from self._issue_s(st, t, kq % self.slots, (ui + 1, 0), n_next[t])
                             early_next[t] = True
                     yield None
-                self.issue(("commit", ("kv_empty", slot_v)))
+                self.commit(("kv_empty", slot_v))
                 if nxt:
-                    self.issue(("commit", ("kv_empty", slot_n)))
+                    self.commit(("kv_empty", slot_n))
+            early = early_next
+
+    def _mma_one_tile(self, t):
+        """Two issuers: this warp issues tile t's MMAs only."""
+        who = 1 + t
+        st = dict(ld=0, qn=[0] * self.nt, pn=[0] * self.nt, on=[0] * self.nt)
+        early = False
+        for ui, n in enumerate(self.units):
+            n_next = self.units[ui + 1] if ui + 1 < len(self.units) else (0,) * self.nt
+            early_next = False
+            nblk = max(n)
+            if nblk == 0:
+                continue
+            ld_unit = st["ld"]
+            slot_k = st["ld"] % self.slots
+            yield self._wait_kv(st, st["ld"])
+            st["ld"] += 1
+            if n[t] and not early:
+                yield from self._issue_s(st, t, slot_k, (ui, 0), n[t], who)
+            self.commit(("kv_empty", slot_k), who)
+            for it in range(nblk):
+                slot_v = st["ld"] % self.slots
+                yield self._wait_kv(st, st["ld"])
+                st["ld"] += 1
+                nxt = it + 1 < nblk
+                ld_n = st["ld"]
+                slot_n = ld_n % self.slots
+                k_ready = False
+                if nxt:
+                    st["ld"] += 1
+                if it < n[t]:
+                    yield from self._issue_pv(st, t, slot_v, (ui, it), who)
+                    if it + 1 < n[t]:
+                        yield self._wait_kv(st, ld_n)
+                        k_ready = True
+                        yield from self._issue_s(st, t, slot_n, (ui, it + 1), n[t], who)
+                    else:
+                        self.commit(("o_full", t), who)
+                        st["on"][t] += 1
+                        rule = 2 * (nblk - it) <= self.slots or "ring_rule" in self.drop
+                        if n_next[t] > 0 and rule:
+                            kq = ld_unit + 2 * nblk
+                            yield self._wait_kv(st, kq)
+                            yield from self._issue_s(st, t, kq % self.slots, (ui + 1, 0),
+                                                     n_next[t], who)
+                            early_next = True
+                yield None
+                self.commit(("kv_empty", slot_v), who)
+                if nxt:
+                    # release K of the next block too, after waiting for it even when this
+                    # tile does not read it: the entry's phase must be the current one
+                    if not k_ready and "every_index" not in self.drop:
+                        yield self._wait_kv(st, ld_n)
+                    self.commit(("kv_empty", slot_n), who)
             early = early_next
 
     def _mma_separate_p(self, st):
@@ -292,7 +370,7 @@ class Cta:
             for t in range(self.nt):
                 if n[t]:
                     yield from self._issue_s(st, t, slot_k, (ui, 0), n[t])
-            self.issue(("commit", ("kv_empty", slot_k)))
+            self.commit(("kv_empty", slot_k))
             for it in range(nblk):
                 slot_v = st["ld"] % self.slots
                 yield self._wait_kv(st, st["ld"])
@@ -308,16 +386,16 @@ class Cta:
                             yield self._wait(("s_free", t), st["sf"][t] & 1)
                         st["sf"][t] += 1
                         yield from self._issue_s(st, t, slot_n, (ui, it + 1), n[t])
-                    self.issue(("commit", ("kv_empty", slot_n)))
+                    self.commit(("kv_empty", slot_n))
                 for t in range(self.nt):
                     if it >= n[t]:
                         continue
                     yield from self._issue_pv(st, t, slot_v, (ui, it))
-                    self.issue(("commit", ("p_free", t)))
+                    self.commit(("p_free", t))
                     if it + 1 == n[t]:
-                        self.issue(("commit", ("o_full", t)))
+                        self.commit(("o_full", t))
                         st["on"][t] += 1
-                self.issue(("commit", ("kv_empty", slot_v)))
+                self.commit(("kv_empty", slot_v))
                 yield None
 
     # ---------------------------------------------------------------- softmax warp
@@ -391,10 +469,11 @@ class Cta:
     def run(self, rng, max_steps=400000):
         """Interleave the actors and the two async engines at random, each with a random
         speed, until everything has finished."""
-        actors = [self.producer(), self.mma()] + ([self.epilogue()] if self.nt == 2 else []) + \
+        mma = [self._mma_one_tile(t) for t in range(self.nt)] if self.two_issuers else [self.mma()]
+        actors = [self.producer()] + mma + ([self.epilogue()] if self.nt == 2 else []) + \
             [self.softmax(t, w) for t in range(self.nt) for w in range(WARPS)]
         na = len(actors)
-        speed = [rng.uniform(0.02, 1.0) for _ in range(na + 2)]  # + tensor pipe, TMA
+        speed = [rng.uniform(0.02, 1.0) for _ in range(na + 3)]  # + tensor pipe, TMA, commits
         cond = [None] * na
         live = list(range(na))
         for _ in range(max_steps):
@@ -403,6 +482,9 @@ class Cta:
                 runnable.append(na)
             if self.tma:
                 runnable.append(na + 1)
+            ready = self.ready_commits()
+            if ready:
+                runnable.append(na + 2)
             if not runnable:
                 if live:
                     raise Deadlock(f"{len(live)} actors blocked with nothing in flight")
@@ -412,6 +494,8 @@ class Cta:
                 self.complete_mma()
             elif i == na + 1:
                 self.complete_tma(rng.randrange(len(self.tma)))
+            elif i == na + 2:
+                self.fire_commit(rng.choice(ready))
             else:
                 try:
                     cond[i] = next(actors[i])
@@ -428,14 +512,14 @@ class Cta:
             raise Race("not every tile's output was read out")
 
 
-def random_cta(rng, separate_p=True, slots=None, drop=(), tiles=2):
+def random_cta(rng, separate_p=True, slots=None, drop=(), tiles=2, two_issuers=False):
     """One to five units per CTA, 0-4 key blocks per tile, random padding-only warps (warp 0
     of a tile with keys always holds a valid row)."""
     units, idle = [], []
     for _ in range(rng.randint(1, 5)):
         units.append(tuple(rng.randint(0, 4) for _ in range(tiles)))
         idle.append([set(w for w in (1, 2, 3) if rng.random() < 0.5) for _ in range(tiles)])
-    return Cta(units, idle, separate_p, slots, drop, tiles)
+    return Cta(units, idle, separate_p, slots, drop, tiles, two_issuers)
 
 
 def run_random(seed, **kw):

@@ -16,6 +16,9 @@ checked on a CPU model under random interleavings (tests/handoff_model.py).
     the LSE) stayed right.
   - Leaving out the ring-position rule of P over S's early first S deadlocks: K_0 of the
     next unit would wait for a ring slot this unit has not released yet.
+* A design under study, one MMA-issuing warp per tile with P over S, is checked the same
+  way before any kernel code: each issuer must walk every ring entry in order, also those
+  its tile does not read, before it releases them (both issuers release every entry).
 * With one tile, two waits are implied by others, and the model shows it:
   - the ring-position rule always holds: the tile ends on its unit's last block;
   - the MMA warp's wait for the released O: the next unit's first P.V already waits for
@@ -28,19 +31,23 @@ import pytest
 from tests import handoff_model as H
 
 SEEDS = range(400)
-# name: (separate P, tiles)
-SCHEDULES = {"two tiles, separate P": (True, 2), "two tiles, P over S": (False, 2),
-             "one tile, P over S": (False, 1)}
+SCHEDULES = {
+    "two tiles, separate P": dict(separate_p=True, tiles=2),
+    "two tiles, P over S": dict(separate_p=False, tiles=2),
+    "one tile, P over S": dict(separate_p=False, tiles=1),
+    # a design under study: one MMA-issuing warp per tile
+    "two tiles, P over S, two issuers": dict(separate_p=False, tiles=2, two_issuers=True),
+}
 ONLY_SEPARATE_P = {"s_free", "p_free", "idle_p_free"}
+ONLY_TWO_ISSUERS = {"every_index"}
 IMPLIED_WITH_ONE_TILE = {"ring_rule", "o_empty"}
 
 
 def outcomes(schedule, drop=()):
-    separate_p, tiles = SCHEDULES[schedule]
     races, deadlocks = [], []
     for seed in SEEDS:
         try:
-            H.run_random(seed, separate_p=separate_p, drop=drop, tiles=tiles)
+            H.run_random(seed, drop=drop, **SCHEDULES[schedule])
         except H.Race as e:
             races.append(str(e))
         except H.Deadlock as e:
@@ -80,12 +87,14 @@ def test_schedule_is_race_and_deadlock_free(schedule):
 
 
 def applies(schedule, wait):
-    separate_p, tiles = SCHEDULES[schedule]
+    kw = SCHEDULES[schedule]
     if wait in ONLY_SEPARATE_P:
-        return separate_p
-    if wait == "ring_rule" and separate_p:
+        return kw["separate_p"]
+    if wait in ONLY_TWO_ISSUERS:
+        return kw.get("two_issuers", False)
+    if wait == "ring_rule" and kw["separate_p"]:
         return False  # the separate-P schedule has no early first S
-    return not (tiles == 1 and wait in IMPLIED_WITH_ONE_TILE)
+    return not (kw["tiles"] == 1 and wait in IMPLIED_WITH_ONE_TILE)
 
 
 CASES = [(s, w) for s in SCHEDULES for w in H.Cta.WAITS if applies(s, w)]
